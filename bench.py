@@ -1,0 +1,411 @@
+#!/usr/bin/env python
+"""Benchmark of the R-SWA decode hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload (default): single-document bf16 decode -- batch 1, 10 heads, head
+dim 128, L_m = 2592 reference rows (10 pages x 256 vision tokens + 32 prompt
+tokens), window n = 128, outputs continuing past T = 6144.  One "step" decodes
+one output token: the fused append+decode kernel runs once for each of R
+layer caches (R distinct caches, as in an R-layer decoder), so the bytes one
+step touches exceed twice the L2 size and nothing is served from L2 between
+steps.  The timed steps start in the steady state (T > n), where the R-SWA
+cost per step is constant and maximal.
+
+value     : tokens/s through one attention layer = B * R * K / device time.
+e2e       : the same through the public binding with HOST buffers: every step
+            copies q, k, v of all R layers from pinned host memory, runs the R
+            calls and copies the outputs back, all inside the timed region.
+roofline  : algorithmic bytes per launch (2 * rows * d * 2 bytes of K and V
+            plus q, o, new k, v) / average launch time, against the measured
+            HBM copy bandwidth.
+
+N > 1 GPUs (one process per GPU under torchrun) run independent replicas of
+the workload (R-SWA shards by sequence with no exchange): value is the sum
+of all ranks' tokens over the slowest rank's time.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "R-SWA decode tokens/s and achieved HBM GB/s (% of B200 peak) vs output length"
+FALLBACK_HBM_GBS = 6650.0
+
+WORKLOADS = {
+    "single_doc": dict(B=1, H=10, d=128, pages=[10], prompt=32, n=128, T=6144, dtype="bf16",
+                       desc="single-document bf16 decode: batch 1, 10 heads, d=128, L_m=2592 "
+                            "(10 pages x 256 + 32), n=128, T=6144"),
+    "ragged": dict(B=64, H=10, d=128, pages=None, prompt=32, n=128, T=6144, dtype="bf16",
+                   desc="ragged batched bf16 decode: 64 sequences, pages~U[2,50], "
+                        "L_m=256*pages+32, 10 heads, d=128, n=128, T=6144"),
+    "long": dict(B=8, H=10, d=128, pages=[50] * 8, prompt=32, n=128, T=100000, dtype="bf16",
+                 desc="long-horizon bf16 decode: batch 8, L_m=12832, 10 heads, d=128, n=128, T=100000"),
+}
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+# ---------------------------------------------------------------- helpers
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for f in ("decode.cu", "common.cuh", "internal.h"):
+        with open(os.path.join(ROOT, "reference_sliding_window_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source for this workload; else None."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "decode_traffic.json")) as f:
+            d = json.load(f)
+        rec = d.get(workload)
+        if rec and rec.get("source_sha") == kernel_source_sha():
+            return float(rec["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [l for l in out.splitlines() if l.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in getattr(self, "lines", []):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------- distributed plumbing
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def reduce_max_sum(elapsed_s: float, units: float, backend_device=None):
+    """Max of the elapsed times and sum of the units over all ranks (a host
+    plumbing reduction, not part of the measured path)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return elapsed_s, units
+    t = torch.tensor([elapsed_s], dtype=torch.float64, device=backend_device)
+    u = torch.tensor([units], dtype=torch.float64, device=backend_device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(u.item())
+
+
+# --------------------------------------------------------------- our arm
+
+def ref_lens_for(w, seed=0):
+    from reference_sliding_window_b200 import synth
+    if w["pages"] is None:
+        pages = synth.ragged_page_counts(w["B"], seed=seed)
+    else:
+        pages = w["pages"]
+    return [synth.reference_length(p, w["prompt"]) for p in pages]
+
+
+def bytes_per_launch(w, lens):
+    s = 2 if w["dtype"] == "bf16" else 4
+    d, H, n = w["d"], w["H"], w["n"]
+    return sum(H * (2 * (L + n) * d * s + 4 * d * s) for L in lens)
+
+
+def run_ours(args, w, lens):
+    import torch
+    import torch.distributed as dist
+    from reference_sliding_window_b200 import RSWA, synth
+
+    world, rank, local = dist_env()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    B, H, d, n = w["B"], w["H"], w["d"], w["n"]
+    dt = synth.torch_dtype(w["dtype"])
+    L_m_cap = max(lens)
+    per_launch = bytes_per_launch(w, lens)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    R = args.layers or max(1, math.ceil(2 * l2 / per_launch))
+
+    # R layer caches with their reference segments
+    layers = []
+    for r in range(R):
+        a = RSWA(L_m_cap, n, H, d, B, dt, device=dev)
+        Kr = synth.normal((B, H, L_m_cap, d), 1000 + r + 7919 * rank, w["dtype"], "cuda")
+        Vr = synth.normal((B, H, L_m_cap, d), 2000 + r + 7919 * rank, w["dtype"], "cuda")
+        a.load_reference(Kr, Vr, lens)
+        del Kr, Vr
+        layers.append(a)
+    P = 16  # distinct per-step inputs, cycled
+    pool = synth.normal((P, R, 3, B, H, d), 3000 + 7919 * rank, w["dtype"], "cuda")
+    out = torch.empty((R, B, H, d), dtype=dt, device=dev)
+
+    def step(i):
+        x = pool[i % P]
+        for r, a in enumerate(layers):
+            a.append_decode(x[r, 0], x[r, 1], x[r, 2], out=out[r])
+
+    stream = torch.cuda.Stream(device=dev)
+    stream.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(stream):
+        # fill the ring (steady state) and warm up
+        for i in range(n + args.warmup):
+            step(i)
+        torch.cuda.synchronize(dev)
+        # capture P steps (R launches each) in one graph
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(P):
+                step(i)
+        for _ in range(max(1, args.warmup // P)):
+            g.replay()
+        torch.cuda.synchronize(dev)
+    reps = max(1, math.ceil(args.steps / P))
+    K = reps * P
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist.is_initialized():
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        start.record(stream)
+        for _ in range(reps):
+            g.replay()
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    if dist.is_initialized():
+        dist.barrier()
+    elapsed = start.elapsed_time(end) / 1e3
+    launches = K * R
+    for a in layers:
+        a.check()
+    T_end = layers[0].step_count()[0]
+
+    # ---- e2e: host buffers through the public binding
+    K_e2e = min(K, max(P, args.e2e_steps))
+    host_in = torch.empty((P, R, 3, B, H, d), dtype=dt, pin_memory=True)
+    host_in.copy_(pool.cpu())
+    host_out = torch.empty((K_e2e, R, B, H, d), dtype=dt, pin_memory=True)
+    dev_in = torch.empty((R, 3, B, H, d), dtype=dt, device=dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for i in range(K_e2e):
+            dev_in.copy_(host_in[i % P], non_blocking=True)
+            for r, a in enumerate(layers):
+                a.append_decode(dev_in[r, 0], dev_in[r, 1], dev_in[r, 2], out=out[r])
+            host_out[i].copy_(out, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+    e2e_s = e0.elapsed_time(e1) / 1e3
+    for a in layers:
+        a.check()
+
+    el_max, tok_sum = reduce_max_sum(elapsed, float(B * R * K), dev)
+    e2e_max, e2e_tok = reduce_max_sum(e2e_s, float(B * R * K_e2e), dev)
+    g.reset()
+    return dict(R=R, K=K, elapsed=elapsed, el_max=el_max, tok_sum=tok_sum, launches=launches,
+                per_launch=per_launch, clocks=clk.summary(), e2e_max=e2e_max, e2e_tok=e2e_tok,
+                K_e2e=K_e2e, T_end=T_end, l2=l2,
+                h2d=int(R * 3 * B * H * d * (2 if w["dtype"] == "bf16" else 4)),
+                d2h=int(R * B * H * d * (2 if w["dtype"] == "bf16" else 4)))
+
+
+# ------------------------------------------------------------ oracle timing
+
+def oracle_sample(w, lens, budget_s: float, seed: int = 0):
+    """Times the fp64 CPU oracle on decode steps of this workload: each
+    sampled step recomputes the attention of one token for every sequence
+    and head from the full history (steady state, T = n + a few).  Returns
+    (tokens/s of one layer, threads, description)."""
+    import numpy as np
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = 1
+    rng = np.random.default_rng(seed)
+    B, H, d, n = w["B"], w["H"], w["d"], w["n"]
+    T = n + 8
+    hist = []
+    for L in lens:
+        Kh = rng.standard_normal((L + T, H, d))
+        Vh = rng.standard_normal((L + T, H, d))
+        hist.append((Kh, Vh))
+    steps, t0 = 0, time.perf_counter()
+    while True:
+        q = rng.standard_normal((H, d))
+        for b, L in enumerate(lens):
+            oracle.decode_step(q, hist[b][0], hist[b][1], L, T, n)
+        steps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s and steps >= 2:
+            break
+    return B * steps / el, threads, f"{steps} decode steps x {B} sequences x {H} heads (T={T}), fp64 numpy"
+
+
+# -------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2048)
+    ap.add_argument("--warmup", type=int, default=16)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="single_doc")
+    ap.add_argument("--layers", type=int, default=0, help="layer caches cycled (0: 2 x L2 rule)")
+    ap.add_argument("--e2e-steps", type=int, default=256)
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle timing")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world, rank, local = dist_env()
+    w = WORKLOADS[args.workload]
+    lens = ref_lens_for(w)
+    config = {"workload": w["desc"], "batch": w["B"], "heads": w["H"], "head_dim": w["d"], "n": w["n"],
+              "L_m": lens if len(lens) <= 8 else {"min": min(lens), "max": max(lens), "mean": sum(lens) / len(lens)}}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        v, threads, sample = oracle_sample(w, lens, args.cpu_budget)
+        line = {"metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": 1e3 * w["B"] / v, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "impl": "reference", "config": dict(config, l2="host CPU"),
+                "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                                 "sample": sample},
+                "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return 0
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        res = run_ours(args, w, lens)
+    finally:
+        pass
+    peak, peak_kind = measured_peaks()
+    avg_launch = res["elapsed"] / res["launches"]
+    achieved = res["per_launch"] / avg_launch / 1e9
+    line = None
+    if rank == 0:
+        cpu = None
+        if world == 1:
+            v, threads, sample = oracle_sample(w, lens, args.cpu_budget)
+            cpu = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample}
+        value = res["tok_sum"] / res["el_max"]
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": res["K"],
+            "warmup": args.warmup, "ms_per_step": 1e3 * res["el_max"] / res["K"], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": w["dtype"], "data": "synthetic",
+            "config": dict(config, layers_cycled=res["R"],
+                           l2=f"inputs larger than L2: {res['R']} layer caches x {res['per_launch'] / 1e6:.2f} MB "
+                              f"= {res['R'] * res['per_launch'] / 1e6:.0f} MB per step vs L2 "
+                              f"{res['l2'] / 1e6:.0f} MB",
+                           T_range=[w["n"] + args.warmup, res["T_end"]],
+                           unit_def="one decode token of one attention layer for one sequence",
+                           parallelism=f"replicas x{world}"),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "peak_kind": f"{peak_kind} HBM copy",
+                         "traffic": recorded_traffic(args.workload),
+                         "algorithmic_bytes_per_launch": res["per_launch"],
+                         "avg_launch_us": avg_launch * 1e6, "kernel": "rswa::decode_kernel<bf16,128,append>"},
+            "clocks": res["clocks"],
+            "e2e": {"value": res["e2e_tok"] / res["e2e_max"], "unit": "tokens/s",
+                    "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"],
+                    "steps": res["K_e2e"]},
+            "gpu_launches": res["launches"],
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,194 @@
+/*
+ * rswa.h -- C ABI of the B200 (sm_100a) Reference Sliding Window Attention
+ * library, librswa.so.
+ *
+ * R-SWA is defined in "Unlimited OCR Works：一篇读懂 R-SWA 如何把长文档 OCR 从
+ * for-loop 推向 one-shot" (WeThinkIn article), 方法展开 §3, Eq.(1)-(4): the
+ * query producing output t attends, with softmax weights
+ * exp(q.k_j / sqrt(d)) normalised over N(t), to
+ *     N(t) = P ∪ D_n(t),  P = {1..L_m},
+ *     D_n(t) = {j | max(L_m+1, L_m+t-n) <= j <= L_m+t-1},
+ * i.e. every reference token (vision tokens + prompt, encoded once and never
+ * updated) and the most recent n outputs.  The decode-side cache therefore
+ * holds C(T) = L_m + min(n, T) <= L_m + n rows (方法展开 §4, Eq.(6)) and is
+ * managed as a fixed-capacity queue that evicts the oldest output
+ * ("多模态文档解析开源新进展:Unlimited OCR技术方案", section
+ * "为什么它能“无限”读下去？关键在 KV cache 恒定").
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Positions in the pages' notation are 1-based; array indices here are
+ *   0-based.  The query that produces output t sits at position L_m+t-1, so
+ *   after T outputs were appended the decode query (the newest output T)
+ *   sees P and outputs max(1, T+1-n)..T, which is L_m + min(n, T) rows.
+ * - MHA: H query heads and H key/value heads.  Head dim d is 64 or 128.
+ * - Element types: RSWA_F32 (float) or RSWA_BF16 (bfloat16).  Accumulation
+ *   is always float32; outputs are written in the input element type.
+ * - scale <= 0 selects 1/sqrt(d) (Eq.(3)).
+ * - Every device buffer is allocated and owned by the caller.  The library
+ *   never allocates device memory; a handle owns host-side metadata only.
+ *   Device pointers must be 16-byte aligned and point at contiguous,
+ *   row-major tensors of the stated shapes.
+ * - Calls are asynchronous on the CUDA stream given at rswa_init (a
+ *   cudaStream_t passed as void*; NULL = the legacy default stream), except
+ *   the query calls marked "synchronous".
+ * - Argument and state errors are detected on the host, return a status and
+ *   launch nothing.  A CUDA launch error returns RSWA_ERR_CUDA.  Anomalies
+ *   only a kernel can see (a bounded wait that timed out, a capacity
+ *   overflow) set a device error word that rswa_check() reports; kernels
+ *   never trap.
+ * - A handle is not thread-safe; distinct handles are independent.
+ *   rswa_last_error() returns a thread-local message for the last failure.
+ */
+#ifndef RSWA_H_
+#define RSWA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  RSWA_OK = 0,
+  RSWA_ERR_ARG = 1,          /* invalid argument (null/misaligned pointer, bad size) */
+  RSWA_ERR_STATE = 2,        /* call not valid in the handle's current state */
+  RSWA_ERR_CAPACITY = 3,     /* would exceed a capacity fixed at rswa_init */
+  RSWA_ERR_UNSUPPORTED = 4,  /* head dim / dtype / device not supported */
+  RSWA_ERR_CUDA = 5,         /* a CUDA runtime call or kernel launch failed */
+  RSWA_ERR_DEVICE = 6        /* a kernel reported an error (see rswa_check) */
+} rswa_status;
+
+typedef enum { RSWA_F32 = 0, RSWA_BF16 = 1 } rswa_dtype;
+
+/* RSWA_MODE_RSWA: the output segment is an n-slot ring, cache L_m + n rows
+ *                 (Eq.(6)).
+ * RSWA_MODE_FULL: full attention over every output (the MHA baseline of
+ *                 Eq.(5)), cache L_m + T_cap rows.  Same kernels, used to
+ *                 show the growing per-step cost the pages compare against
+ *                 (方法展开 §5, Fig.3). */
+typedef enum { RSWA_MODE_RSWA = 0, RSWA_MODE_FULL = 1 } rswa_mode;
+
+typedef struct rswa_ctx* rswa_handle;
+
+/* ------------------------------------------------------------------------
+ * Sizing.  Pure host functions; no device needed.
+ *
+ * window_cap is n for RSWA_MODE_RSWA and T_cap (the maximum number of
+ * outputs) for RSWA_MODE_FULL.  Returns 0 for invalid arguments.
+ * ---------------------------------------------------------------------- */
+
+/* Bytes of ONE of the two cache tensors (K or V):
+ * [batch][H][L_m_cap + window_cap][d] elements of dtype. */
+size_t rswa_cache_bytes(int L_m_cap, int window_cap, int H, int d, int batch,
+                        rswa_dtype dtype);
+
+/* Bytes of the device workspace (step counters, reference lengths, launch
+ * plan, split-K partials and tickets).  Must be passed to rswa_init. */
+size_t rswa_workspace_bytes(int L_m_cap, int window_cap, int H, int d, int batch);
+
+/* ------------------------------------------------------------------------
+ * Decode-side state.
+ * ---------------------------------------------------------------------- */
+
+/* Creates a handle over caller-owned device memory.
+ *   k_cache, v_cache: rswa_cache_bytes(...) each.  Layout
+ *     [batch][H][L_m_cap + window_cap][d]: for sequence b, rows
+ *     [0, L_m[b]) hold the reference segment and rows
+ *     [L_m[b], L_m[b] + window_cap) the output segment (the n-slot ring in
+ *     RSWA mode, outputs in order in FULL mode).
+ *   workspace: rswa_workspace_bytes(...) bytes; zeroed by this call
+ *     (stream-ordered).
+ *   n: window size (RSWA mode, >= 1).  T_cap: max outputs (FULL mode, >= 1).
+ *   The other of n / T_cap is ignored.
+ * Requires a CUDA device of compute capability 10.0 (B200). */
+rswa_status rswa_init(rswa_handle* out, rswa_mode mode, int L_m_cap, int n, int T_cap,
+                      int H, int d, int batch, rswa_dtype dtype,
+                      void* k_cache, void* v_cache, void* workspace,
+                      size_t workspace_bytes, void* stream);
+
+/* Loads the reference segment ("encoded once and never updated") and
+ * resets every sequence to T = 0 outputs.
+ *   K_ref, V_ref: device [batch][H][ref_stride][d] (row r of (b, h) at
+ *     ((b*H + h)*ref_stride + r)*d); rows [0, ref_lens[b]) are copied.
+ *   ref_lens: HOST array [batch], 1 <= ref_lens[b] <= min(L_m_cap, ref_stride). */
+rswa_status rswa_load_reference(rswa_handle h, const void* K_ref, const void* V_ref,
+                                int ref_stride, const int32_t* ref_lens);
+
+/* Appends output T+1 of every sequence: k, v device [batch][H][d].  In RSWA
+ * mode the row goes to ring slot (T mod n), overwriting the oldest output
+ * once the ring is full (the queue's "position m+1"); in FULL mode to row
+ * L_m + T.  Then T := T+1 (on the device). */
+rswa_status rswa_append(rswa_handle h, const void* k, const void* v);
+
+/* Decode attention of the current step: q, o device [batch][H][d].  Attends
+ * to the L_m[b] + min(n, T[b]) cached rows (FULL: L_m[b] + T[b]).  Split-K
+ * over the cache rows, float32 online softmax, log-sum-exp combine. */
+rswa_status rswa_decode(rswa_handle h, const void* q, void* o, float scale);
+
+/* rswa_append followed by rswa_decode in ONE kernel: the new k, v are
+ * written in place into their slot (no compaction copy) while the cache is
+ * streamed, and the step counter is advanced on the device, so a captured
+ * CUDA graph of this call can be replayed step after step. */
+rswa_status rswa_append_decode(rswa_handle h, const void* k, const void* v,
+                               const void* q, void* o, float scale);
+
+/* Synchronous: cache occupancy L_m[b] + min(n, T[b]) (FULL: L_m[b] + T[b])
+ * per sequence, Eq.(6) / Eq.(5).  out: HOST int32[batch]. */
+rswa_status rswa_cache_len(rswa_handle h, int32_t* out);
+
+/* Synchronous: number of outputs T[b] appended so far.  out: HOST int32[batch]. */
+rswa_status rswa_step_count(rswa_handle h, int32_t* out);
+
+/* Synchronous: the logical 1-based position held by each valid cache row of
+ * sequence b, in storage order (reference rows 1..L_m first, then the
+ * output rows).  out: HOST int64[capacity]; *count receives the number of
+ * rows (= rswa_cache_len()[b]).  RSWA_ERR_CAPACITY if capacity is short. */
+rswa_status rswa_cache_positions(rswa_handle h, int b, int64_t* out, int capacity,
+                                 int* count);
+
+/* Stream-ordered: T := 0 for every sequence; the reference rows are kept. */
+rswa_status rswa_reset(rswa_handle h);
+
+/* Changes the stream later calls are issued on. */
+rswa_status rswa_set_stream(rswa_handle h, void* stream);
+
+/* Synchronous: RSWA_ERR_DEVICE if a kernel raised the device error word
+ * since the last check (the word is then cleared), else RSWA_OK.  The
+ * message names the condition. */
+rswa_status rswa_check(rswa_handle h);
+
+/* Frees the handle's host metadata.  Device buffers stay the caller's. */
+void rswa_destroy(rswa_handle h);
+
+/* ------------------------------------------------------------------------
+ * Teacher-forced (packed prefill / training) form.
+ *
+ * O = softmax(Q K^T * scale + M) V per head, with M = 0 where key j is
+ * visible from query p and -inf elsewhere:
+ *   p <= L_m : j <= p                       (causal inside the prefix)
+ *   p >  L_m : j <= L_m, or p-n+1 <= j <= p  (Eq.(1)-(2) with t = p-L_m+1)
+ * Q, K, V, O: device [L][H][d] (token-major).  1 <= L_m <= L, n >= 1.
+ * BF16 runs on the tcgen05 tensor-core kernel (d = 128), F32 on a SIMT
+ * kernel (d = 64 or 128).  Tiles the mask fully hides are skipped.
+ * ---------------------------------------------------------------------- */
+rswa_status rswa_masked_forward(const void* Q, const void* K, const void* V, void* O,
+                                int L, int L_m, int n, int H, int d, rswa_dtype dtype,
+                                float scale, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Misc.
+ * ---------------------------------------------------------------------- */
+
+/* Thread-local description of the last non-OK status (never NULL). */
+const char* rswa_last_error(void);
+
+/* Library version string, e.g. "rswa 0.1.0 sm_100a". */
+const char* rswa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RSWA_H_ */

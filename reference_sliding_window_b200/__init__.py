@@ -1,0 +1,201 @@
+"""B200 (sm_100a) Reference Sliding Window Attention.
+
+Thin Python binding over the C ABI of librswa.so (include/rswa.h).  It only
+checks and marshals arguments: torch tensors supply device memory and the
+current CUDA stream; every step of the attention runs in the library's CUDA
+kernels.  If the library is missing or the device is not a B200 the calls
+raise; nothing is computed any other way.
+
+    attn = RSWA(L_m_cap=2592, n=128, H=10, d=128, batch=1, dtype=torch.bfloat16)
+    attn.load_reference(K_ref, V_ref, ref_lens)        # [B, H, L_m_cap, d]
+    o = attn.append_decode(k, v, q)                    # [B, H, d] each
+    O = masked_forward(Q, K, V, L_m=..., n=128)        # [L, H, d]
+"""
+
+from __future__ import annotations
+
+import ctypes as C
+from typing import Optional, Sequence
+
+import numpy as np
+import torch
+
+from . import _native
+from ._native import MODE_FULL, MODE_RSWA, RSWAError, check
+
+__all__ = ["RSWA", "masked_forward", "RSWAError", "MODE_RSWA", "MODE_FULL", "library_version"]
+
+_DT = {torch.float32: _native.F32, torch.bfloat16: _native.BF16}
+
+
+def library_version() -> str:
+    return _native.lib().rswa_version().decode()
+
+
+def _stream_ptr(device: torch.device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _check_tensor(name: str, t: torch.Tensor, shape, dtype, device) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+class RSWA:
+    """Decode-side R-SWA state over caller-owned device memory.
+
+    The K/V caches ([B, H, L_m_cap + window, d] each) and the workspace are
+    torch tensors owned by this object; the library itself allocates
+    nothing.  mode MODE_RSWA keeps an n-slot output ring (cache L_m + n);
+    MODE_FULL keeps every output (cache L_m + T_cap), the full-attention
+    baseline.
+    """
+
+    def __init__(self, L_m_cap: int, n: int, H: int, d: int, batch: int,
+                 dtype: torch.dtype = torch.bfloat16, mode: int = MODE_RSWA, T_cap: int = 0,
+                 device: Optional[torch.device] = None):
+        if dtype not in _DT:
+            raise ValueError(f"dtype {dtype} not supported (float32, bfloat16)")
+        dev = torch.device(device) if device is not None else torch.device("cuda")
+        if dev.type != "cuda":
+            raise ValueError(f"RSWA needs a CUDA device, got {dev}")
+        if dev.index is None:
+            dev = torch.device("cuda", torch.cuda.current_device())
+        self.device = dev
+        self.L_m_cap, self.n, self.H, self.d, self.batch = L_m_cap, n, H, d, batch
+        self.dtype, self.mode, self.T_cap = dtype, mode, T_cap
+        self.window = n if mode == MODE_RSWA else T_cap
+        L = _native.lib()
+        cache_bytes = L.rswa_cache_bytes(L_m_cap, self.window, H, d, batch, _DT[dtype])
+        ws_bytes = L.rswa_workspace_bytes(L_m_cap, self.window, H, d, batch)
+        if cache_bytes == 0 or ws_bytes == 0:
+            raise ValueError("invalid sizes for RSWA")
+        self.S_cap = L_m_cap + self.window
+        self.k_cache = torch.zeros((batch, H, self.S_cap, d), dtype=dtype, device=self.device)
+        self.v_cache = torch.zeros((batch, H, self.S_cap, d), dtype=dtype, device=self.device)
+        self.workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=self.device)
+        self._stream = _stream_ptr(self.device)
+        h = C.c_void_p()
+        with torch.cuda.device(self.device):
+            check(L.rswa_init(C.byref(h), mode, L_m_cap, n, T_cap, H, d, batch, _DT[dtype],
+                              self.k_cache.data_ptr(), self.v_cache.data_ptr(),
+                              self.workspace.data_ptr(), ws_bytes, self._stream))
+        self._h = h
+
+    # -- plumbing
+    def _sync_stream(self) -> None:
+        s = _stream_ptr(self.device)
+        if s != self._stream:
+            check(_native.lib().rswa_set_stream(self._h, s))
+            self._stream = s
+
+    def _vec(self, name, t):
+        _check_tensor(name, t, (self.batch, self.H, self.d), self.dtype, self.device)
+
+    def close(self) -> None:
+        if getattr(self, "_h", None):
+            _native.lib().rswa_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # -- API
+    def load_reference(self, K_ref: torch.Tensor, V_ref: torch.Tensor, ref_lens: Sequence[int]) -> None:
+        """K_ref, V_ref: [B, H, stride, d] on the device; rows [0, ref_lens[b]) are used."""
+        if K_ref.dim() != 4:
+            raise ValueError("K_ref must be [B, H, stride, d]")
+        stride = K_ref.shape[2]
+        _check_tensor("K_ref", K_ref, (self.batch, self.H, stride, self.d), self.dtype, self.device)
+        _check_tensor("V_ref", V_ref, (self.batch, self.H, stride, self.d), self.dtype, self.device)
+        lens = (C.c_int32 * self.batch)(*[int(x) for x in ref_lens])
+        if len(ref_lens) != self.batch:
+            raise ValueError("ref_lens must have one entry per sequence")
+        self._sync_stream()
+        check(_native.lib().rswa_load_reference(self._h, K_ref.data_ptr(), V_ref.data_ptr(), stride, lens))
+
+    def append(self, k: torch.Tensor, v: torch.Tensor) -> None:
+        self._vec("k", k)
+        self._vec("v", v)
+        self._sync_stream()
+        check(_native.lib().rswa_append(self._h, k.data_ptr(), v.data_ptr()))
+
+    def decode(self, q: torch.Tensor, out: Optional[torch.Tensor] = None, scale: float = 0.0) -> torch.Tensor:
+        self._vec("q", q)
+        o = torch.empty_like(q) if out is None else out
+        self._vec("out", o)
+        self._sync_stream()
+        check(_native.lib().rswa_decode(self._h, q.data_ptr(), o.data_ptr(), float(scale)))
+        return o
+
+    def append_decode(self, k: torch.Tensor, v: torch.Tensor, q: torch.Tensor,
+                      out: Optional[torch.Tensor] = None, scale: float = 0.0) -> torch.Tensor:
+        self._vec("k", k)
+        self._vec("v", v)
+        self._vec("q", q)
+        o = torch.empty_like(q) if out is None else out
+        self._vec("out", o)
+        self._sync_stream()
+        check(_native.lib().rswa_append_decode(self._h, k.data_ptr(), v.data_ptr(), q.data_ptr(),
+                                               o.data_ptr(), float(scale)))
+        return o
+
+    def cache_len(self) -> list:
+        out = (C.c_int32 * self.batch)()
+        self._sync_stream()
+        check(_native.lib().rswa_cache_len(self._h, out))
+        return list(out)
+
+    def step_count(self) -> list:
+        out = (C.c_int32 * self.batch)()
+        self._sync_stream()
+        check(_native.lib().rswa_step_count(self._h, out))
+        return list(out)
+
+    def cache_positions(self, b: int) -> np.ndarray:
+        cap = self.S_cap
+        out = (C.c_int64 * cap)()
+        cnt = C.c_int()
+        self._sync_stream()
+        check(_native.lib().rswa_cache_positions(self._h, int(b), out, cap, C.byref(cnt)))
+        return np.frombuffer(out, dtype=np.int64, count=cnt.value).copy()
+
+    def reset(self) -> None:
+        self._sync_stream()
+        check(_native.lib().rswa_reset(self._h))
+
+    def check(self) -> None:
+        """Raises RSWAError if a kernel flagged a device-side error."""
+        self._sync_stream()
+        check(_native.lib().rswa_check(self._h))
+
+
+def masked_forward(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, L_m: int, n: int,
+                   scale: float = 0.0, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Teacher-forced R-SWA attention.  Q, K, V, out: [L, H, d] on a B200."""
+    if Q.dim() != 3:
+        raise ValueError("Q must be [L, H, d]")
+    L, H, d = Q.shape
+    if Q.dtype not in _DT:
+        raise ValueError(f"dtype {Q.dtype} not supported")
+    for name, t in (("K", K), ("V", V)):
+        _check_tensor(name, t, (L, H, d), Q.dtype, Q.device)
+    _check_tensor("Q", Q, (L, H, d), Q.dtype, Q.device)
+    O = torch.empty_like(Q) if out is None else out
+    _check_tensor("out", O, (L, H, d), Q.dtype, Q.device)
+    with torch.cuda.device(Q.device):
+        check(_native.lib().rswa_masked_forward(Q.data_ptr(), K.data_ptr(), V.data_ptr(), O.data_ptr(),
+                                                L, int(L_m), int(n), H, d, _DT[Q.dtype], float(scale),
+                                                _stream_ptr(Q.device)))
+    return O

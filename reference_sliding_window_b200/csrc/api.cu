@@ -1,0 +1,549 @@
+// C ABI of librswa (declared in include/rswa.h): argument and state
+// validation, the workspace layout, the split-K launch planner and the
+// kernel launches.  Host code only; every step of the attention runs in the
+// kernels of decode.cu, append.cu and the masked-forward files.
+
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <string>
+#include <vector>
+
+#include "internal.h"
+#include "rswa.h"
+
+using namespace rswa;
+
+// ------------------------------------------------------------------ errors
+
+static thread_local std::string g_last_error = "no error";
+
+static rswa_status fail(rswa_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+static rswa_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(RSWA_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+#define RSWA_CUDA(call, what)              \
+  do {                                     \
+    cudaError_t e_ = (call);               \
+    if (e_ != cudaSuccess) return cuda_fail(e_, what); \
+  } while (0)
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static int elem_size(rswa_dtype t) { return t == RSWA_BF16 ? 2 : 4; }
+
+static bool dtype_ok(rswa_dtype t) { return t == RSWA_F32 || t == RSWA_BF16; }
+
+// ------------------------------------------------------------- workspace
+
+namespace rswa {
+
+static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Split-K partials are bounded: the planner never makes more items than
+// B*H (one per (b, h)) plus kExtraItems.
+static constexpr int kExtraItems = 4096;
+
+WorkspaceLayout workspace_layout(int B, int H, int d) {
+  WorkspaceLayout w{};
+  size_t off = 0;
+  w.err = off;
+  w.done = off + 4;
+  off = 256;
+  w.T = off;
+  off = align_up(off + 4 * (size_t)B, 256);
+  w.Lm = off;
+  off = align_up(off + 4 * (size_t)B, 256);
+  w.tickets = off;
+  off = align_up(off + 4 * (size_t)B * H, 256);
+  w.items_cap = B * H + kExtraItems;
+  w.items = off;
+  off = align_up(off + sizeof(DecodeItem) * (size_t)w.items_cap, 256);
+  w.partials = off;
+  off = align_up(off + 4 * (size_t)(d + 4) * w.items_cap, 256);
+  w.total = off;
+  return w;
+}
+
+}  // namespace rswa
+
+// ------------------------------------------------------------------ handle
+
+struct rswa_ctx {
+  rswa_mode mode;
+  int L_m_cap, n, T_cap, H, d, B;
+  rswa_dtype dtype;
+  int window_cap, S_cap, row_bytes;
+  int device, num_sms;
+  void* kc;
+  void* vc;
+  uint8_t* ws;
+  cudaStream_t stream;
+  WorkspaceLayout lay;
+  bool loaded;
+  int T_host;                 // outputs appended so far (same for every b)
+  std::vector<int32_t> Lm;    // host copy of the reference lengths
+  int plan_window;            // output rows the current plan covers
+  int chunk, n_items;
+  std::vector<DecodeItem> items;
+};
+
+static int32_t* ws_i32(rswa_ctx* c, size_t off) { return reinterpret_cast<int32_t*>(c->ws + off); }
+
+static rswa_status check_handle(rswa_handle h) {
+  if (!h) return fail(RSWA_ERR_ARG, "null handle");
+  return RSWA_OK;
+}
+
+static rswa_status use_device(rswa_ctx* c) {
+  int cur = -1;
+  RSWA_CUDA(cudaGetDevice(&cur), "cudaGetDevice");
+  if (cur != c->device) RSWA_CUDA(cudaSetDevice(c->device), "cudaSetDevice");
+  return RSWA_OK;
+}
+
+// Cost model of the split-K planner: a CTA streams its items one after the
+// other; an item costs its rows plus a fixed per-item overhead (epilogue
+// and merge) expressed in rows.
+static constexpr int kItemOverheadRows = 16;
+
+// Chooses the rows-per-item `chunk` minimising the slowest CTA's work under
+// static round-robin assignment, then lays out the items.
+static void make_plan(rswa_ctx* c) {
+  const int G = c->num_sms;
+  std::vector<int> rows(c->B);
+  int max_rows = 0;
+  for (int b = 0; b < c->B; ++b) {
+    rows[b] = std::min(c->Lm[b] + c->plan_window, c->S_cap);
+    max_rows = std::max(max_rows, rows[b]);
+  }
+  long long best_cost = -1;
+  int best_chunk = 32;
+  const int top = std::max(32, (max_rows + 31) / 32 * 32);
+  for (int C = 32; C <= top; C += 32) {
+    long long items = 0;
+    for (int b = 0; b < c->B; ++b) items += (long long)c->H * ((rows[b] + C - 1) / C);
+    if (items > c->lay.items_cap) continue;
+    const long long waves = (items + G - 1) / G;
+    const long long cost = waves * (long long)(C + kItemOverheadRows);
+    if (best_cost < 0 || cost <= best_cost) {
+      best_cost = cost;
+      best_chunk = C;
+    }
+  }
+  c->chunk = best_chunk;
+  c->items.clear();
+  int part = 0;
+  for (int b = 0; b < c->B; ++b) {
+    const int np = (rows[b] + best_chunk - 1) / best_chunk;
+    for (int h = 0; h < c->H; ++h) {
+      for (int k = 0; k < np; ++k) {
+        DecodeItem it;
+        it.bh = b * c->H + h;
+        it.row0 = k * best_chunk;
+        it.part = part + k;
+        it.nparts = np;
+        c->items.push_back(it);
+      }
+      part += np;
+    }
+  }
+  c->n_items = (int)c->items.size();
+}
+
+static rswa_status upload_plan(rswa_ctx* c) {
+  RSWA_CUDA(cudaMemcpyAsync(c->ws + c->lay.items, c->items.data(),
+                            sizeof(DecodeItem) * c->items.size(), cudaMemcpyHostToDevice,
+                            c->stream),
+            "upload decode plan");
+  return RSWA_OK;
+}
+
+// FULL mode: the plan must cover the rows of the next step.
+static rswa_status ensure_plan(rswa_ctx* c, int T_next) {
+  if (c->mode == RSWA_MODE_RSWA) return RSWA_OK;
+  if (T_next <= c->plan_window) return RSWA_OK;
+  c->plan_window = std::min(c->T_cap, (T_next + 511) / 512 * 512);
+  make_plan(c);
+  return upload_plan(c);
+}
+
+// ------------------------------------------------------------------ sizing
+
+extern "C" size_t rswa_cache_bytes(int L_m_cap, int window_cap, int H, int d, int batch,
+                                   rswa_dtype dtype) {
+  if (L_m_cap < 1 || window_cap < 1 || H < 1 || batch < 1 || (d != 64 && d != 128) ||
+      !dtype_ok(dtype))
+    return 0;
+  return (size_t)batch * H * (size_t)(L_m_cap + window_cap) * d * elem_size(dtype);
+}
+
+extern "C" size_t rswa_workspace_bytes(int L_m_cap, int window_cap, int H, int d, int batch) {
+  if (L_m_cap < 1 || window_cap < 1 || H < 1 || batch < 1 || (d != 64 && d != 128)) return 0;
+  return workspace_layout(batch, H, d).total;
+}
+
+// ---------------------------------------------------------------- lifetime
+
+extern "C" rswa_status rswa_init(rswa_handle* out, rswa_mode mode, int L_m_cap, int n, int T_cap,
+                                 int H, int d, int batch, rswa_dtype dtype, void* k_cache,
+                                 void* v_cache, void* workspace, size_t workspace_bytes,
+                                 void* stream) {
+  if (!out) return fail(RSWA_ERR_ARG, "rswa_init: out is null");
+  *out = nullptr;
+  if (mode != RSWA_MODE_RSWA && mode != RSWA_MODE_FULL)
+    return fail(RSWA_ERR_ARG, "rswa_init: unknown mode %d", (int)mode);
+  if (!dtype_ok(dtype)) return fail(RSWA_ERR_UNSUPPORTED, "rswa_init: unknown dtype %d", (int)dtype);
+  if (d != 64 && d != 128) return fail(RSWA_ERR_UNSUPPORTED, "rswa_init: head dim %d (64 or 128)", d);
+  if (L_m_cap < 1 || H < 1 || batch < 1)
+    return fail(RSWA_ERR_ARG, "rswa_init: L_m_cap=%d H=%d batch=%d must be >= 1", L_m_cap, H, batch);
+  if (mode == RSWA_MODE_RSWA && n < 1) return fail(RSWA_ERR_ARG, "rswa_init: window n=%d must be >= 1", n);
+  if (mode == RSWA_MODE_FULL && T_cap < 1)
+    return fail(RSWA_ERR_ARG, "rswa_init: T_cap=%d must be >= 1 in FULL mode", T_cap);
+  const int window_cap = mode == RSWA_MODE_RSWA ? n : T_cap;
+  if ((long long)L_m_cap + window_cap > (1ll << 30))
+    return fail(RSWA_ERR_ARG, "rswa_init: L_m_cap + window too large");
+  if (!k_cache || !v_cache || !workspace) return fail(RSWA_ERR_ARG, "rswa_init: null buffer");
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(workspace))
+    return fail(RSWA_ERR_ARG, "rswa_init: buffers must be 16-byte aligned");
+  const WorkspaceLayout lay = workspace_layout(batch, H, d);
+  if (workspace_bytes < lay.total)
+    return fail(RSWA_ERR_ARG, "rswa_init: workspace of %zu bytes, need %zu", workspace_bytes, lay.total);
+
+  int dev = 0;
+  RSWA_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  cudaDeviceProp prop;
+  RSWA_CUDA(cudaGetDeviceProperties(&prop, dev), "cudaGetDeviceProperties");
+  if (prop.major != 10 || prop.minor != 0)
+    return fail(RSWA_ERR_UNSUPPORTED, "rswa_init: device %d is sm_%d%d; this library is built for sm_100a",
+                dev, prop.major, prop.minor);
+  const size_t smem = decode_smem_bytes(dtype == RSWA_BF16 ? kBF16 : kF32, d);
+  if ((size_t)prop.sharedMemPerBlockOptin < smem)
+    return fail(RSWA_ERR_UNSUPPORTED, "rswa_init: kernel needs %zu bytes of shared memory", smem);
+
+  rswa_ctx* c = new rswa_ctx();
+  c->mode = mode;
+  c->L_m_cap = L_m_cap;
+  c->n = n;
+  c->T_cap = T_cap;
+  c->H = H;
+  c->d = d;
+  c->B = batch;
+  c->dtype = dtype;
+  c->window_cap = window_cap;
+  c->S_cap = L_m_cap + window_cap;
+  c->row_bytes = d * elem_size(dtype);
+  c->device = dev;
+  c->num_sms = prop.multiProcessorCount;
+  c->kc = k_cache;
+  c->vc = v_cache;
+  c->ws = static_cast<uint8_t*>(workspace);
+  c->stream = static_cast<cudaStream_t>(stream);
+  c->lay = lay;
+  c->loaded = false;
+  c->T_host = 0;
+  c->plan_window = 0;
+  c->chunk = 32;
+  c->n_items = 0;
+  cudaError_t e = cudaMemsetAsync(c->ws, 0, lay.total, c->stream);
+  if (e != cudaSuccess) {
+    delete c;
+    return cuda_fail(e, "rswa_init: clear workspace");
+  }
+  *out = c;
+  return RSWA_OK;
+}
+
+extern "C" void rswa_destroy(rswa_handle h) { delete h; }
+
+extern "C" rswa_status rswa_set_stream(rswa_handle h, void* stream) {
+  if (rswa_status st = check_handle(h)) return st;
+  h->stream = static_cast<cudaStream_t>(stream);
+  return RSWA_OK;
+}
+
+// ----------------------------------------------------------------- reference
+
+extern "C" rswa_status rswa_load_reference(rswa_handle h, const void* K_ref, const void* V_ref,
+                                           int ref_stride, const int32_t* ref_lens) {
+  if (rswa_status st = check_handle(h)) return st;
+  if (!K_ref || !V_ref || !ref_lens) return fail(RSWA_ERR_ARG, "rswa_load_reference: null argument");
+  if (!aligned16(K_ref) || !aligned16(V_ref))
+    return fail(RSWA_ERR_ARG, "rswa_load_reference: K_ref/V_ref must be 16-byte aligned");
+  if (ref_stride < 1) return fail(RSWA_ERR_ARG, "rswa_load_reference: ref_stride=%d", ref_stride);
+  int max_len = 0;
+  for (int b = 0; b < h->B; ++b) {
+    const int L = ref_lens[b];
+    if (L < 1 || L > h->L_m_cap || L > ref_stride)
+      return fail(RSWA_ERR_CAPACITY, "rswa_load_reference: ref_lens[%d]=%d outside [1, min(L_m_cap=%d, ref_stride=%d)]",
+                  b, L, h->L_m_cap, ref_stride);
+    max_len = std::max(max_len, L);
+  }
+  if (rswa_status st = use_device(h)) return st;
+  h->Lm.assign(ref_lens, ref_lens + h->B);
+  h->T_host = 0;
+  h->plan_window = h->mode == RSWA_MODE_RSWA ? h->n : std::min(h->T_cap, 512);
+  make_plan(h);
+  RSWA_CUDA(cudaMemcpyAsync(h->ws + h->lay.Lm, h->Lm.data(), 4 * (size_t)h->B, cudaMemcpyHostToDevice,
+                            h->stream),
+            "upload reference lengths");
+  RSWA_CUDA(cudaMemsetAsync(h->ws + h->lay.T, 0, 4 * (size_t)h->B, h->stream), "reset step counters");
+  if (rswa_status st = upload_plan(h)) return st;
+  LoadRefParams p;
+  p.kc = h->kc;
+  p.vc = h->vc;
+  p.K_ref = K_ref;
+  p.V_ref = V_ref;
+  p.B = h->B;
+  p.H = h->H;
+  p.S_cap = h->S_cap;
+  p.row_bytes = h->row_bytes;
+  p.ref_stride = ref_stride;
+  p.Lm = ws_i32(h, h->lay.Lm);
+  RSWA_CUDA(launch_load_reference(p, max_len, h->stream), "load_reference kernel");
+  h->loaded = true;
+  return RSWA_OK;
+}
+
+// ------------------------------------------------------------------- steps
+
+static rswa_status check_step(rswa_ctx* c, bool appending, const char* who) {
+  if (!c->loaded) return fail(RSWA_ERR_STATE, "%s: call rswa_load_reference first", who);
+  if (appending && c->mode == RSWA_MODE_FULL && c->T_host + 1 > c->T_cap)
+    return fail(RSWA_ERR_CAPACITY, "%s: FULL mode holds at most T_cap=%d outputs", who, c->T_cap);
+  return RSWA_OK;
+}
+
+extern "C" rswa_status rswa_append(rswa_handle h, const void* k, const void* v) {
+  if (rswa_status st = check_handle(h)) return st;
+  if (!k || !v) return fail(RSWA_ERR_ARG, "rswa_append: null k/v");
+  if (!aligned16(k) || !aligned16(v)) return fail(RSWA_ERR_ARG, "rswa_append: k/v must be 16-byte aligned");
+  if (rswa_status st = check_step(h, true, "rswa_append")) return st;
+  if (rswa_status st = use_device(h)) return st;
+  if (rswa_status st = ensure_plan(h, h->T_host + 1)) return st;
+  AppendParams p;
+  p.kc = h->kc;
+  p.vc = h->vc;
+  p.k_new = k;
+  p.v_new = v;
+  p.B = h->B;
+  p.H = h->H;
+  p.S_cap = h->S_cap;
+  p.row_bytes = h->row_bytes;
+  p.n = h->n;
+  p.full_mode = h->mode == RSWA_MODE_FULL;
+  p.T_cap = h->T_cap;
+  p.T = ws_i32(h, h->lay.T);
+  p.Lm = ws_i32(h, h->lay.Lm);
+  p.err = ws_i32(h, h->lay.err);
+  RSWA_CUDA(launch_append(p, h->stream), "append kernel");
+  h->T_host += 1;
+  return RSWA_OK;
+}
+
+static rswa_status run_decode(rswa_ctx* c, const void* k, const void* v, const void* q, void* o,
+                              float scale, bool append, const char* who) {
+  if (!q || !o) return fail(RSWA_ERR_ARG, "%s: null q/o", who);
+  if (!aligned16(q) || !aligned16(o)) return fail(RSWA_ERR_ARG, "%s: q/o must be 16-byte aligned", who);
+  if (append) {
+    if (!k || !v) return fail(RSWA_ERR_ARG, "%s: null k/v", who);
+    if (!aligned16(k) || !aligned16(v)) return fail(RSWA_ERR_ARG, "%s: k/v must be 16-byte aligned", who);
+  }
+  if (!(scale == scale) || isinf(scale)) return fail(RSWA_ERR_ARG, "%s: scale is not finite", who);
+  if (rswa_status st = check_step(c, append, who)) return st;
+  if (rswa_status st = use_device(c)) return st;
+  if (rswa_status st = ensure_plan(c, c->T_host + (append ? 1 : 0))) return st;
+  DecodeParams p;
+  p.kc = c->kc;
+  p.vc = c->vc;
+  p.kc_w = c->kc;
+  p.vc_w = c->vc;
+  p.q = q;
+  p.o = o;
+  p.k_new = k;
+  p.v_new = v;
+  p.B = c->B;
+  p.H = c->H;
+  p.S_cap = c->S_cap;
+  p.n = c->n;
+  p.full_mode = c->mode == RSWA_MODE_FULL;
+  p.T_cap = c->T_cap;
+  p.chunk = c->chunk;
+  p.n_items = c->n_items;
+  p.T = ws_i32(c, c->lay.T);
+  p.Lm = ws_i32(c, c->lay.Lm);
+  p.items = reinterpret_cast<const DecodeItem*>(c->ws + c->lay.items);
+  p.partials = reinterpret_cast<float*>(c->ws + c->lay.partials);
+  p.tickets = ws_i32(c, c->lay.tickets);
+  p.done = ws_i32(c, c->lay.done);
+  p.err = ws_i32(c, c->lay.err);
+  const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)c->d);
+  p.scale_log2 = sc * 1.4426950408889634f;
+  const int grid = std::min(c->n_items, c->num_sms);
+  RSWA_CUDA(launch_decode(c->dtype == RSWA_BF16 ? kBF16 : kF32, c->d, append, p, grid, c->stream),
+            "decode kernel");
+  if (append) c->T_host += 1;
+  return RSWA_OK;
+}
+
+extern "C" rswa_status rswa_decode(rswa_handle h, const void* q, void* o, float scale) {
+  if (rswa_status st = check_handle(h)) return st;
+  return run_decode(h, nullptr, nullptr, q, o, scale, false, "rswa_decode");
+}
+
+extern "C" rswa_status rswa_append_decode(rswa_handle h, const void* k, const void* v, const void* q,
+                                          void* o, float scale) {
+  if (rswa_status st = check_handle(h)) return st;
+  return run_decode(h, k, v, q, o, scale, true, "rswa_append_decode");
+}
+
+// ----------------------------------------------------------------- queries
+
+static rswa_status read_T(rswa_ctx* c, std::vector<int32_t>& T) {
+  if (rswa_status st = use_device(c)) return st;
+  T.assign(c->B, 0);
+  RSWA_CUDA(cudaMemcpyAsync(T.data(), c->ws + c->lay.T, 4 * (size_t)c->B, cudaMemcpyDeviceToHost,
+                            c->stream),
+            "read step counters");
+  RSWA_CUDA(cudaStreamSynchronize(c->stream), "cudaStreamSynchronize");
+  // Graph replays advance the device counters without the host; follow them.
+  c->T_host = T.empty() ? 0 : T[0];
+  return RSWA_OK;
+}
+
+extern "C" rswa_status rswa_step_count(rswa_handle h, int32_t* out) {
+  if (rswa_status st = check_handle(h)) return st;
+  if (!out) return fail(RSWA_ERR_ARG, "rswa_step_count: null out");
+  if (!h->loaded) return fail(RSWA_ERR_STATE, "rswa_step_count: no reference loaded");
+  std::vector<int32_t> T;
+  if (rswa_status st = read_T(h, T)) return st;
+  memcpy(out, T.data(), 4 * (size_t)h->B);
+  return RSWA_OK;
+}
+
+static int occupancy(const rswa_ctx* c, int b, int T) {
+  return c->mode == RSWA_MODE_RSWA ? c->Lm[b] + std::min(c->n, T) : c->Lm[b] + T;
+}
+
+extern "C" rswa_status rswa_cache_len(rswa_handle h, int32_t* out) {
+  if (rswa_status st = check_handle(h)) return st;
+  if (!out) return fail(RSWA_ERR_ARG, "rswa_cache_len: null out");
+  if (!h->loaded) return fail(RSWA_ERR_STATE, "rswa_cache_len: no reference loaded");
+  std::vector<int32_t> T;
+  if (rswa_status st = read_T(h, T)) return st;
+  for (int b = 0; b < h->B; ++b) out[b] = occupancy(h, b, T[b]);
+  return RSWA_OK;
+}
+
+extern "C" rswa_status rswa_cache_positions(rswa_handle h, int b, int64_t* out, int capacity,
+                                            int* count) {
+  if (rswa_status st = check_handle(h)) return st;
+  if (!out || !count) return fail(RSWA_ERR_ARG, "rswa_cache_positions: null out/count");
+  if (!h->loaded) return fail(RSWA_ERR_STATE, "rswa_cache_positions: no reference loaded");
+  if (b < 0 || b >= h->B) return fail(RSWA_ERR_ARG, "rswa_cache_positions: b=%d outside [0, %d)", b, h->B);
+  std::vector<int32_t> T;
+  if (rswa_status st = read_T(h, T)) return st;
+  const int Tb = T[b];
+  const int rows = occupancy(h, b, Tb);
+  *count = rows;
+  if (capacity < rows) return fail(RSWA_ERR_CAPACITY, "rswa_cache_positions: need %d entries", rows);
+  const int Lm = h->Lm[b];
+  for (int r = 0; r < Lm; ++r) out[r] = r + 1;
+  if (h->mode == RSWA_MODE_FULL) {
+    for (int j = 1; j <= Tb; ++j) out[Lm + j - 1] = (int64_t)Lm + j;
+  } else {
+    // Ring slot s holds the newest output j <= T with (j - 1) mod n == s.
+    const int used = std::min(h->n, Tb);
+    for (int s = 0; s < used; ++s) {
+      const int back = ((Tb - 1 - s) % h->n + h->n) % h->n;
+      out[Lm + s] = (int64_t)Lm + (Tb - back);
+    }
+  }
+  return RSWA_OK;
+}
+
+extern "C" rswa_status rswa_reset(rswa_handle h) {
+  if (rswa_status st = check_handle(h)) return st;
+  if (!h->loaded) return fail(RSWA_ERR_STATE, "rswa_reset: no reference loaded");
+  if (rswa_status st = use_device(h)) return st;
+  RSWA_CUDA(cudaMemsetAsync(h->ws + h->lay.T, 0, 4 * (size_t)h->B, h->stream), "reset step counters");
+  h->T_host = 0;
+  return RSWA_OK;
+}
+
+extern "C" rswa_status rswa_check(rswa_handle h) {
+  if (rswa_status st = check_handle(h)) return st;
+  if (rswa_status st = use_device(h)) return st;
+  int32_t err = 0;
+  RSWA_CUDA(cudaMemcpyAsync(&err, h->ws + h->lay.err, 4, cudaMemcpyDeviceToHost, h->stream),
+            "read device error word");
+  RSWA_CUDA(cudaStreamSynchronize(h->stream), "cudaStreamSynchronize");
+  if (err == 0) return RSWA_OK;
+  RSWA_CUDA(cudaMemsetAsync(h->ws + h->lay.err, 0, 4, h->stream), "clear device error word");
+  std::string what;
+  if (err & kErrWaitTimeout) what += " wait-timeout";
+  if (err & kErrPlanShort) what += " plan-short";
+  if (err & kErrCapacity) what += " capacity";
+  if (err & kErrTmemAlloc) what += " tmem-alloc";
+  return fail(RSWA_ERR_DEVICE, "device error word 0x%x:%s", err, what.c_str());
+}
+
+// ---------------------------------------------------------- masked forward
+
+extern "C" rswa_status rswa_masked_forward(const void* Q, const void* K, const void* V, void* O, int L,
+                                           int L_m, int n, int H, int d, rswa_dtype dtype, float scale,
+                                           void* stream) {
+  if (!Q || !K || !V || !O) return fail(RSWA_ERR_ARG, "rswa_masked_forward: null tensor");
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
+    return fail(RSWA_ERR_ARG, "rswa_masked_forward: tensors must be 16-byte aligned");
+  if (!dtype_ok(dtype)) return fail(RSWA_ERR_UNSUPPORTED, "rswa_masked_forward: unknown dtype");
+  if (d != 64 && d != 128) return fail(RSWA_ERR_UNSUPPORTED, "rswa_masked_forward: head dim %d", d);
+  if (L < 1 || H < 1) return fail(RSWA_ERR_ARG, "rswa_masked_forward: L=%d H=%d", L, H);
+  if (L_m < 1 || L_m > L) return fail(RSWA_ERR_ARG, "rswa_masked_forward: L_m=%d outside [1, L=%d]", L_m, L);
+  if (n < 1) return fail(RSWA_ERR_ARG, "rswa_masked_forward: n=%d must be >= 1", n);
+  if (!(scale == scale) || isinf(scale)) return fail(RSWA_ERR_ARG, "rswa_masked_forward: scale not finite");
+  if ((long long)L * H * d >= (1ll << 31))
+    return fail(RSWA_ERR_ARG, "rswa_masked_forward: tensor too large");
+  int dev = 0;
+  RSWA_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  int major = 0, minor = 0;
+  RSWA_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev), "device attribute");
+  RSWA_CUDA(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev), "device attribute");
+  if (major != 10 || minor != 0)
+    return fail(RSWA_ERR_UNSUPPORTED, "rswa_masked_forward: device is sm_%d%d; built for sm_100a", major, minor);
+  MaskedParams p;
+  p.Q = Q;
+  p.K = K;
+  p.V = V;
+  p.O = O;
+  p.L = L;
+  p.L_m = L_m;
+  p.n = n;
+  p.H = H;
+  p.D = d;
+  const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)d);
+  p.scale_log2 = sc * 1.4426950408889634f;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  RSWA_CUDA(launch_masked_forward_simt(p, dtype == RSWA_BF16 ? kBF16 : kF32, s), "masked forward kernel");
+  return RSWA_OK;
+}
+
+// -------------------------------------------------------------------- misc
+
+extern "C" const char* rswa_last_error(void) { return g_last_error.c_str(); }
+
+extern "C" const char* rswa_version(void) { return "rswa 0.1.0 sm_100a"; }
