@@ -109,7 +109,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
         time.sleep(0.3)
@@ -239,17 +239,18 @@ def run_ours(args, w, lens):
     reps = max(1, math.ceil(args.steps / P))
     K = reps * P
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if dist.is_initialized():
-        dist.barrier()
-    torch.cuda.synchronize(dev)
-    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
-        start.record(stream)
-        for _ in range(reps):
-            g.replay()
-        end.record(stream)
+    with torch.cuda.stream(stream):  # graph replays launch on the current stream
+        if dist.is_initialized():
+            dist.barrier()
         torch.cuda.synchronize(dev)
-    if dist.is_initialized():
-        dist.barrier()
+        with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+            start.record(stream)
+            for _ in range(reps):
+                g.replay()
+            end.record(stream)
+            torch.cuda.synchronize(dev)
+        if dist.is_initialized():
+            dist.barrier()
     elapsed = start.elapsed_time(end) / 1e3
     launches = K * R
     for a in layers:
@@ -326,7 +327,7 @@ def oracle_sample(w, lens, budget_s: float, seed: int = 0):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2048)
+    ap.add_argument("--steps", type=int, default=6144)
     ap.add_argument("--warmup", type=int, default=16)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="single_doc")

@@ -54,9 +54,9 @@ namespace rswa {
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// Split-K partials are bounded: the planner never makes more items than
-// B*H (one per (b, h)) plus kExtraItems.
-static constexpr int kExtraItems = 4096;
+// Split-K partials are bounded: a span plan has at most one item per slab
+// plus one per CTA boundary.
+static constexpr int kMaxCtas = 1024;
 
 WorkspaceLayout workspace_layout(int B, int H, int d) {
   WorkspaceLayout w{};
@@ -65,14 +65,17 @@ WorkspaceLayout workspace_layout(int B, int H, int d) {
   w.done = off + 4;
   off = 256;
   w.T = off;
-  off = align_up(off + 4 * (size_t)B, 256);
+  off = align_up(off + 4, 256);
   w.Lm = off;
   off = align_up(off + 4 * (size_t)B, 256);
   w.tickets = off;
   off = align_up(off + 4 * (size_t)B * H, 256);
-  w.items_cap = B * H + kExtraItems;
+  w.max_ctas = kMaxCtas;
+  w.items_cap = B * H + kMaxCtas;
   w.items = off;
   off = align_up(off + sizeof(DecodeItem) * (size_t)w.items_cap, 256);
+  w.cta_begin = off;
+  off = align_up(off + 4 * (size_t)(kMaxCtas + 1), 256);
   w.partials = off;
   off = align_up(off + 4 * (size_t)(d + 4) * w.items_cap, 256);
   w.total = off;
@@ -98,8 +101,9 @@ struct rswa_ctx {
   int T_host;                 // outputs appended so far (same for every b)
   std::vector<int32_t> Lm;    // host copy of the reference lengths
   int plan_window;            // output rows the current plan covers
-  int chunk, n_items;
+  int n_ctas;
   std::vector<DecodeItem> items;
+  std::vector<int32_t> cta_begin;
 };
 
 static int32_t* ws_i32(rswa_ctx* c, size_t off) { return reinterpret_cast<int32_t*>(c->ws + off); }
@@ -116,59 +120,69 @@ static rswa_status use_device(rswa_ctx* c) {
   return RSWA_OK;
 }
 
-// Cost model of the split-K planner: a CTA streams its items one after the
-// other; an item costs its rows plus a fixed per-item overhead (epilogue
-// and merge) expressed in rows.
-static constexpr int kItemOverheadRows = 16;
-
-// Chooses the rows-per-item `chunk` minimising the slowest CTA's work under
-// static round-robin assignment, then lays out the items.
+// Span planner: the planned rows of every (b, h) slab (b-major, then h) are
+// laid end to end in 32-row stages and cut into G nearly equal contiguous
+// spans, one per CTA, G = min(#SMs, #stages).  A span splits into items at
+// slab boundaries, so every CTA streams the same number of stages (+-1) and
+// a slab is merged from only as many partials as spans that touch it.
 static void make_plan(rswa_ctx* c) {
-  const int G = c->num_sms;
-  std::vector<int> rows(c->B);
-  int max_rows = 0;
+  const int nbh = c->B * c->H;
+  std::vector<int> rows(nbh), stages(nbh);
+  long long total = 0;
   for (int b = 0; b < c->B; ++b) {
-    rows[b] = std::min(c->Lm[b] + c->plan_window, c->S_cap);
-    max_rows = std::max(max_rows, rows[b]);
-  }
-  long long best_cost = -1;
-  int best_chunk = 32;
-  const int top = std::max(32, (max_rows + 31) / 32 * 32);
-  for (int C = 32; C <= top; C += 32) {
-    long long items = 0;
-    for (int b = 0; b < c->B; ++b) items += (long long)c->H * ((rows[b] + C - 1) / C);
-    if (items > c->lay.items_cap) continue;
-    const long long waves = (items + G - 1) / G;
-    const long long cost = waves * (long long)(C + kItemOverheadRows);
-    if (best_cost < 0 || cost <= best_cost) {
-      best_cost = cost;
-      best_chunk = C;
-    }
-  }
-  c->chunk = best_chunk;
-  c->items.clear();
-  int part = 0;
-  for (int b = 0; b < c->B; ++b) {
-    const int np = (rows[b] + best_chunk - 1) / best_chunk;
+    const int r = std::min(c->Lm[b] + c->plan_window, c->S_cap);
     for (int h = 0; h < c->H; ++h) {
-      for (int k = 0; k < np; ++k) {
-        DecodeItem it;
-        it.bh = b * c->H + h;
-        it.row0 = k * best_chunk;
-        it.part = part + k;
-        it.nparts = np;
-        c->items.push_back(it);
-      }
-      part += np;
+      rows[b * c->H + h] = r;
+      stages[b * c->H + h] = (r + 31) / 32;
+      total += (r + 31) / 32;
     }
   }
-  c->n_items = (int)c->items.size();
+  const int G = (int)std::min<long long>(std::min(c->num_sms, c->lay.max_ctas), total);
+  c->items.clear();
+  c->cta_begin.assign(G + 1, 0);
+  std::vector<int> first_item(nbh, -1), count(nbh, 0);
+  int bh = 0, st_in_bh = 0;  // walk position: slab and stage inside it
+  for (int g = 0; g < G; ++g) {
+    c->cta_begin[g] = (int)c->items.size();
+    long long todo = (total * (g + 1)) / G - (total * g) / G;  // stages of this span
+    while (todo > 0) {
+      const int take = (int)std::min<long long>(todo, stages[bh] - st_in_bh);
+      DecodeItem it{};
+      it.bh = bh;
+      it.row0 = st_in_bh * 32;
+      it.rows = std::min(rows[bh], (st_in_bh + take) * 32) - it.row0;
+      it.last = (st_in_bh + take == stages[bh]) ? 1 : 0;
+      if (first_item[bh] < 0) first_item[bh] = (int)c->items.size();
+      count[bh] += 1;
+      c->items.push_back(it);
+      todo -= take;
+      st_in_bh += take;
+      if (st_in_bh == stages[bh]) {
+        ++bh;
+        st_in_bh = 0;
+      }
+    }
+  }
+  c->cta_begin[G] = (int)c->items.size();
+  // Partials: item i is partial i; each slab's items are consecutive.
+  for (size_t i = 0; i < c->items.size(); ++i) {
+    DecodeItem& it = c->items[i];
+    it.part = (int)i;
+    it.part_first = first_item[it.bh];
+    it.nparts = count[it.bh];
+  }
+  c->n_ctas = G;
 }
 
 static rswa_status upload_plan(rswa_ctx* c) {
+  if ((int)c->items.size() > c->lay.items_cap)
+    return fail(RSWA_ERR_CAPACITY, "decode plan of %zu items exceeds %d", c->items.size(), c->lay.items_cap);
   RSWA_CUDA(cudaMemcpyAsync(c->ws + c->lay.items, c->items.data(),
                             sizeof(DecodeItem) * c->items.size(), cudaMemcpyHostToDevice,
                             c->stream),
+            "upload decode plan");
+  RSWA_CUDA(cudaMemcpyAsync(c->ws + c->lay.cta_begin, c->cta_begin.data(),
+                            sizeof(int32_t) * c->cta_begin.size(), cudaMemcpyHostToDevice, c->stream),
             "upload decode plan");
   return RSWA_OK;
 }
@@ -177,7 +191,7 @@ static rswa_status upload_plan(rswa_ctx* c) {
 static rswa_status ensure_plan(rswa_ctx* c, int T_next) {
   if (c->mode == RSWA_MODE_RSWA) return RSWA_OK;
   if (T_next <= c->plan_window) return RSWA_OK;
-  c->plan_window = std::min(c->T_cap, (T_next + 511) / 512 * 512);
+  c->plan_window = std::min(c->T_cap, (T_next + 63) / 64 * 64);
   make_plan(c);
   return upload_plan(c);
 }
@@ -257,8 +271,7 @@ extern "C" rswa_status rswa_init(rswa_handle* out, rswa_mode mode, int L_m_cap, 
   c->loaded = false;
   c->T_host = 0;
   c->plan_window = 0;
-  c->chunk = 32;
-  c->n_items = 0;
+  c->n_ctas = 0;
   cudaError_t e = cudaMemsetAsync(c->ws, 0, lay.total, c->stream);
   if (e != cudaSuccess) {
     delete c;
@@ -296,12 +309,12 @@ extern "C" rswa_status rswa_load_reference(rswa_handle h, const void* K_ref, con
   if (rswa_status st = use_device(h)) return st;
   h->Lm.assign(ref_lens, ref_lens + h->B);
   h->T_host = 0;
-  h->plan_window = h->mode == RSWA_MODE_RSWA ? h->n : std::min(h->T_cap, 512);
+  h->plan_window = h->mode == RSWA_MODE_RSWA ? h->n : std::min(h->T_cap, 64);
   make_plan(h);
   RSWA_CUDA(cudaMemcpyAsync(h->ws + h->lay.Lm, h->Lm.data(), 4 * (size_t)h->B, cudaMemcpyHostToDevice,
                             h->stream),
             "upload reference lengths");
-  RSWA_CUDA(cudaMemsetAsync(h->ws + h->lay.T, 0, 4 * (size_t)h->B, h->stream), "reset step counters");
+  RSWA_CUDA(cudaMemsetAsync(h->ws + h->lay.T, 0, 4, h->stream), "reset step counter");
   if (rswa_status st = upload_plan(h)) return st;
   LoadRefParams p;
   p.kc = h->kc;
@@ -355,6 +368,12 @@ extern "C" rswa_status rswa_append(rswa_handle h, const void* k, const void* v) 
   return RSWA_OK;
 }
 
+// Profiling aid: per-CTA timestamp buffer used by RSWA_TIMING builds.
+static unsigned long long* g_timing = nullptr;
+#ifdef RSWA_TIMING
+extern "C" void rswa_debug_set_timing(void* buf) { g_timing = static_cast<unsigned long long*>(buf); }
+#endif
+
 static rswa_status run_decode(rswa_ctx* c, const void* k, const void* v, const void* q, void* o,
                               float scale, bool append, const char* who) {
   if (!q || !o) return fail(RSWA_ERR_ARG, "%s: null q/o", who);
@@ -382,18 +401,20 @@ static rswa_status run_decode(rswa_ctx* c, const void* k, const void* v, const v
   p.n = c->n;
   p.full_mode = c->mode == RSWA_MODE_FULL;
   p.T_cap = c->T_cap;
-  p.chunk = c->chunk;
-  p.n_items = c->n_items;
+  p.n_ctas = c->n_ctas;
+  p.n_items_total = (int)c->items.size();
   p.T = ws_i32(c, c->lay.T);
   p.Lm = ws_i32(c, c->lay.Lm);
   p.items = reinterpret_cast<const DecodeItem*>(c->ws + c->lay.items);
+  p.cta_begin = reinterpret_cast<const int32_t*>(c->ws + c->lay.cta_begin);
   p.partials = reinterpret_cast<float*>(c->ws + c->lay.partials);
   p.tickets = ws_i32(c, c->lay.tickets);
   p.done = ws_i32(c, c->lay.done);
   p.err = ws_i32(c, c->lay.err);
   const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)c->d);
   p.scale_log2 = sc * 1.4426950408889634f;
-  const int grid = std::min(c->n_items, c->num_sms);
+  p.timing = g_timing;
+  const int grid = c->n_ctas;
   RSWA_CUDA(launch_decode(c->dtype == RSWA_BF16 ? kBF16 : kF32, c->d, append, p, grid, c->stream),
             "decode kernel");
   if (append) c->T_host += 1;
@@ -413,15 +434,15 @@ extern "C" rswa_status rswa_append_decode(rswa_handle h, const void* k, const vo
 
 // ----------------------------------------------------------------- queries
 
+// The device step counter is one int: every sequence advances together.
 static rswa_status read_T(rswa_ctx* c, std::vector<int32_t>& T) {
   if (rswa_status st = use_device(c)) return st;
-  T.assign(c->B, 0);
-  RSWA_CUDA(cudaMemcpyAsync(T.data(), c->ws + c->lay.T, 4 * (size_t)c->B, cudaMemcpyDeviceToHost,
-                            c->stream),
-            "read step counters");
+  int32_t t = 0;
+  RSWA_CUDA(cudaMemcpyAsync(&t, c->ws + c->lay.T, 4, cudaMemcpyDeviceToHost, c->stream), "read step counter");
   RSWA_CUDA(cudaStreamSynchronize(c->stream), "cudaStreamSynchronize");
-  // Graph replays advance the device counters without the host; follow them.
-  c->T_host = T.empty() ? 0 : T[0];
+  // Graph replays advance the device counter without the host; follow it.
+  c->T_host = t;
+  T.assign(c->B, t);
   return RSWA_OK;
 }
 
@@ -480,7 +501,7 @@ extern "C" rswa_status rswa_reset(rswa_handle h) {
   if (rswa_status st = check_handle(h)) return st;
   if (!h->loaded) return fail(RSWA_ERR_STATE, "rswa_reset: no reference loaded");
   if (rswa_status st = use_device(h)) return st;
-  RSWA_CUDA(cudaMemsetAsync(h->ws + h->lay.T, 0, 4 * (size_t)h->B, h->stream), "reset step counters");
+  RSWA_CUDA(cudaMemsetAsync(h->ws + h->lay.T, 0, 4, h->stream), "reset step counter");
   h->T_host = 0;
   return RSWA_OK;
 }

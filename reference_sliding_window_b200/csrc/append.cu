@@ -14,32 +14,29 @@
 
 namespace rswa {
 
-// One CTA per sequence b: read T once, write the H new rows of k and v,
-// then advance T.  No other CTA touches T[b], so there is no race.
+// One CTA: read the step counter T once, write the B*H new rows of k and v
+// into their slots, then advance T.  Only this CTA touches T, so there is no
+// race.  (Not the hot path: decoding uses the fused kernel.)
 __global__ void __launch_bounds__(256) append_kernel(const __grid_constant__ AppendParams p) {
-  __shared__ int s_slot, s_T;
-  const int b = blockIdx.x;
+  __shared__ int s_T, s_ok;
   if (threadIdx.x == 0) {
-    const int Tn = __ldcg(p.T + b) + 1;
-    int slot;
-    if (p.full_mode) {
-      slot = (Tn <= p.T_cap) ? p.Lm[b] + Tn - 1 : -1;
-      if (slot < 0) flag_error(p.err, kErrCapacity);
-    } else {
-      slot = p.Lm[b] + (Tn - 1) % p.n;
-    }
-    s_slot = slot;
+    const int Tn = __ldcg(p.T) + 1;
+    const int ok = !p.full_mode || Tn <= p.T_cap;
+    if (!ok) flag_error(p.err, kErrCapacity);
     s_T = Tn;
+    s_ok = ok;
   }
   __syncthreads();
-  const int slot = s_slot;
-  if (slot >= 0) {
+  const int Tn = s_T;
+  if (s_ok) {
     const int vpr = p.row_bytes / 16;
-    for (int i = threadIdx.x; i < p.H * vpr; i += blockDim.x) {
-      const int h = i / vpr, c = i % vpr;
-      const size_t bh = (size_t)b * p.H + h;
-      const size_t src = bh * p.row_bytes + (size_t)c * 16;
-      const size_t dst = (bh * p.S_cap + slot) * p.row_bytes + (size_t)c * 16;
+    const long long total = (long long)p.B * p.H * vpr;
+    for (long long i = threadIdx.x; i < total; i += blockDim.x) {
+      const int bh = (int)(i / vpr), c = (int)(i % vpr);
+      const int b = bh / p.H;
+      const int slot = p.full_mode ? p.Lm[b] + Tn - 1 : p.Lm[b] + (Tn - 1) % p.n;
+      const size_t src = (size_t)bh * p.row_bytes + (size_t)c * 16;
+      const size_t dst = ((size_t)bh * p.S_cap + slot) * p.row_bytes + (size_t)c * 16;
       *reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.kc) + dst) =
           *reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.k_new) + src);
       *reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.vc) + dst) =
@@ -47,7 +44,7 @@ __global__ void __launch_bounds__(256) append_kernel(const __grid_constant__ App
     }
   }
   __syncthreads();
-  if (threadIdx.x == 0 && slot >= 0) p.T[b] = s_T;
+  if (threadIdx.x == 0 && s_ok) *p.T = Tn;
 }
 
 // grid.y = B*H slabs, grid.x covers max_len rows x vectors; copies rows
@@ -70,7 +67,7 @@ __global__ void __launch_bounds__(256) load_reference_kernel(const __grid_consta
 }
 
 cudaError_t launch_append(const AppendParams& p, cudaStream_t stream) {
-  append_kernel<<<p.B, 256, 0, stream>>>(p);
+  append_kernel<<<1, 256, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

@@ -10,8 +10,8 @@
 
 namespace rswa {
 
-// A bounded wait gives up after this many nanoseconds of global time.
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
+// A bounded wait gives up after this many SM clock cycles (about 2 s).
+constexpr long long kWaitLimitCycles = 4000000000ll;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -55,13 +55,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Waits until the phase with the given parity has completed.  Returns false
-// (and the caller must flag kErrWaitTimeout and stop) after kWaitLimitNs.
+// (and the caller must flag kErrWaitTimeout and stop) after kWaitLimitCycles.
+// The bound uses the SM-local cycle counter, read once per 64 tries.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = global_ns();
+  const long long t0 = clock64();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (global_ns() - t0 > kWaitLimitNs) return false;
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (clock64() - t0 > kWaitLimitCycles) return false;
   }
 }
 
@@ -73,6 +75,11 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst_smem, const void* src, uin
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
       ::"r"(dst_smem), "l"(src), "r"(bytes), "r"(bar)
       : "memory");
+}
+
+// Bulk prefetch of global memory into L2 (no shared-memory destination).
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 __device__ __forceinline__ void named_barrier_sync(int id, int threads) {

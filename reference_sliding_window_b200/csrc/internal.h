@@ -17,27 +17,34 @@ enum DeviceError : int {
 };
 
 
-// One unit of decode work: a run of up to `chunk` cache rows of one (b, h).
-//   bh:        b * H + h
-//   row0:      first cache row of the run
-//   part:      index of this item's split-K partial
-//   nparts:    number of items (= partials) of this (b, h); its partials are
-//              part - row0/chunk ... + nparts - 1
+// One unit of decode work: a run of cache rows of one (b, h) slab, processed
+// by one CTA.  Each CTA owns a contiguous range of items (a span of the
+// concatenated slabs), so a CTA has at most a few items and a slab is split
+// over at most a few CTAs.
+//   bh:          b * H + h
+//   row0, rows:  first cache row and planned row count (a multiple of 32
+//                except at the end of the slab)
+//   part:        index of this item's split-K partial
+//   part_first, nparts: the partials of this (b, h)
+//   last:        1 if this item ends the planned rows of its slab
 struct DecodeItem {
-  int32_t bh, row0, part, nparts;
+  int32_t bh, row0, rows, part;
+  int32_t part_first, nparts, last, pad;
 };
 
 // Device workspace layout (byte offsets from the workspace base).
 struct WorkspaceLayout {
   size_t err;        // int32: device error word
   size_t done;       // int32: end-of-launch ticket (fused append+decode)
-  size_t T;          // int32[B]: outputs appended so far
+  size_t T;          // int32: outputs appended so far (every sequence advances together)
   size_t Lm;         // int32[B]: reference rows
   size_t tickets;    // int32[B*H]: split-K tickets
   size_t items;      // DecodeItem[items_cap]
+  size_t cta_begin;  // int32[max_ctas + 1]: first item of each CTA
   size_t partials;   // float[items_cap][d + 4]: (o[0..d), m, l, pad)
   size_t total;
   int items_cap;
+  int max_ctas;
 };
 
 WorkspaceLayout workspace_layout(int B, int H, int d);
@@ -57,16 +64,18 @@ struct DecodeParams {
   int n;                 // ring size (RSWA mode)
   int full_mode;         // 0: ring of n slots, 1: outputs in order
   int T_cap;             // FULL mode capacity
-  int chunk;             // rows per item (multiple of 32)
-  int n_items;
-  int32_t* T;            // [B]
+  int n_ctas;            // grid size; CTA c runs items [cta_begin[c], cta_begin[c+1])
+  int n_items_total;
+  int32_t* T;            // scalar step counter
   const int32_t* Lm;     // [B]
   const DecodeItem* items;
+  const int32_t* cta_begin;
   float* partials;
   int32_t* tickets;
   int32_t* done;
   int32_t* err;
   float scale_log2;      // softmax scale * log2(e)
+  unsigned long long* timing;  // profiling stamps (RSWA_TIMING builds), may be null
 };
 
 // Launch the split-K decode kernel (append: fused ring write + T advance).

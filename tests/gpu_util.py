@@ -58,6 +58,9 @@ def run_steps(a: RSWA, case: synth.DecodeCase, steps, sample=None, fused: bool =
             o = a.decode(q[t - 1])
         if sample is None or t in sample:
             outs[t] = o.clone()
+        if t % 512 == 0:  # localise any device-side error to a window of steps
+            torch.cuda.synchronize()
+            a.check()
     torch.cuda.synchronize()
     a.check()
     return outs

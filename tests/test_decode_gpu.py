@@ -121,7 +121,7 @@ def test_full_mode_and_its_capacity():
 
 
 def test_full_mode_replans_past_first_window():
-    # FULL mode plans 512 output rows at a time; cross that boundary.
+    # FULL mode plans 64 output rows at a time; cross several boundaries.
     case = synth.decode_case(B=1, H=2, d=64, ref_lens=[30], n=8, T=530, dtype="f32", seed=8)
     a = make_attn(case, mode=MODE_FULL, T_cap=600)
     outs = run_steps(a, case, case.T, sample={1, 511, 512, 513, 530})
