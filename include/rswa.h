@@ -178,6 +178,36 @@ rswa_status rswa_masked_forward(const void* Q, const void* K, const void* V, voi
                                 float scale, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Decode without allocation.  The pages have no counterpart to this call;
+ * it exists for callers that cannot allocate device memory: a plugin inside
+ * a host framework that owns every device allocation, code that must avoid
+ * the implicitly synchronising cudaMalloc / cudaFree, or code running while
+ * a stream is being captured, where allocation calls are not permitted.
+ *
+ * One-shot decode attention over caller-owned caches, with no handle and no
+ * workspace: the kernel's scratch (launch plan, split-K partials, tickets)
+ * lives in a static device array of about 0.7 MB inside the library, which
+ * every device that loads the library holds until the process exits.  The
+ * library allocates nothing for this call.
+ *   k_cache, v_cache: device [batch][H][S_cap][d]; for (b, h), rows
+ *     [0, cache_lens[b]) are attended, in any storage order (for example
+ *     the reference rows followed by the ring of an RSWA handle).
+ *   cache_lens: HOST int32[batch], 1 <= cache_lens[b] <= S_cap.
+ *   q, o: device [batch][H][d].  scale <= 0 selects 1/sqrt(d).
+ * Limits: batch * H <= 1024; d = 64 or 128.  Larger sizes return
+ * RSWA_ERR_CAPACITY with a message in rswa_last_error().
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  Every call reuses the same array and clears
+ * what must start at zero, so calls whose kernels overlap on the GPU race:
+ * order them on one stream.  Kernel-side error flags are not reported.
+ * ---------------------------------------------------------------------- */
+rswa_status rswa_decode_noalloc(const void* k_cache, const void* v_cache, int S_cap,
+                                const int32_t* cache_lens, const void* q, void* o,
+                                int batch, int H, int d, rswa_dtype dtype, float scale,
+                                void* stream);
+
+/* ------------------------------------------------------------------------
  * Misc.
  * ---------------------------------------------------------------------- */
 

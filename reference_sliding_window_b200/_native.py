@@ -35,6 +35,7 @@ _PROTOS = {
     "rswa_check": (_i, [_p]),
     "rswa_destroy": (None, [_p]),
     "rswa_masked_forward": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _p]),
+    "rswa_decode_noalloc": (_i, [_p, _p, _i, C.POINTER(C.c_int32), _p, _p, _i, _i, _i, _i, _f, _p]),
     "rswa_last_error": (C.c_char_p, []),
     "rswa_version": (C.c_char_p, []),
 }

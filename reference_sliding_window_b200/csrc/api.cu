@@ -32,6 +32,10 @@ static rswa_status fail(rswa_status st, const char* fmt, ...) {
   return st;
 }
 
+void rswa::set_last_error(const char* prefix, const char* msg) {
+  g_last_error = std::string(prefix) + msg;
+}
+
 static rswa_status cuda_fail(cudaError_t e, const char* what) {
   return fail(RSWA_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
 }

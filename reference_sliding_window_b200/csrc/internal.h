@@ -114,6 +114,9 @@ struct MaskedParams {
   int L, L_m, n, H, D;
   float scale_log2;
 };
+// Sets the thread-local message returned by rswa_last_error().
+void set_last_error(const char* prefix, const char* msg);
+
 cudaError_t launch_masked_forward_simt(const MaskedParams& p, int elem, cudaStream_t stream);
 
 }  // namespace rswa
