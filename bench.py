@@ -56,11 +56,25 @@ WORKLOADS = {
 }
 
 
+PREFILL = dict(L=32768, L_m=12832, n=128, H=10, d=128, dtype="bf16",
+               desc="teacher-forced masked prefill, bf16: packed 32768-token sequence, 10 heads, d=128, "
+                    "L_m=12832 reference tokens + 19936 outputs, n=128")
+
+
+def visible_pairs(L, L_m, n):
+    """Visible (query, key) pairs per head of the packed R-SWA mask."""
+    T_out = L - L_m
+    return L_m * (L_m + 1) // 2 + T_out * L_m + sum(min(n, t) for t in range(1, T_out + 1))
+
+
 def log(*a):
     print(*a, file=sys.stderr, flush=True)
 
 
 # ---------------------------------------------------------------- helpers
+
+FALLBACK_BF16_TFLOPS = 1590.0
+
 
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -70,6 +84,49 @@ def measured_peaks():
         return float(d["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def measured_tensor_peak():
+    """Dense bf16 TFLOP/s: the burst figure (a kernel timed on its own)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def run_prefill(iters: int, warmup: int):
+    """Times rswa_masked_forward on the 32K teacher-forced config (inputs
+    252 MB, larger than L2).  Returns a dict for the JSON line."""
+    import torch
+    from reference_sliding_window_b200 import masked_forward, synth
+    w = PREFILL
+    dev = torch.device("cuda", torch.cuda.current_device())
+    Q, K, V = synth.prefill_case(w["L"], w["H"], w["d"], w["dtype"], seed=21, device="cuda")
+    O = torch.empty_like(Q)
+    for _ in range(max(1, warmup)):
+        masked_forward(Q, K, V, L_m=w["L_m"], n=w["n"], out=O)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(iters):
+        masked_forward(Q, K, V, L_m=w["L_m"], n=w["n"], out=O)
+    e1.record()
+    torch.cuda.synchronize(dev)
+    sec = e0.elapsed_time(e1) / 1e3 / iters
+    pairs = visible_pairs(w["L"], w["L_m"], w["n"])
+    flops = 4.0 * w["d"] * pairs * w["H"]
+    dense_causal = 4.0 * w["d"] * (w["L"] * (w["L"] + 1) // 2) * w["H"]
+    peak, kind = measured_tensor_peak()
+    tf = flops / sec / 1e12
+    return {"workload": w["desc"], "ms_per_call": sec * 1e3, "iters": iters,
+            "tflops": tf, "visible_pairs_per_head": pairs,
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
+                         "frac": tf / peak, "peak_kind": f"{kind} dense bf16 (burst)",
+                         "traffic": None, "algorithmic_flops_per_launch": flops,
+                         "kernel": "rswa::tc::masked_tc_kernel"},
+            "dense_causal_flops": dense_causal}
 
 
 def kernel_source_sha() -> str:
@@ -330,7 +387,8 @@ def main():
     ap.add_argument("--steps", type=int, default=6144)
     ap.add_argument("--warmup", type=int, default=16)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="single_doc")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["prefill"], default="single_doc")
+    ap.add_argument("--prefill-iters", type=int, default=10, help="timed masked-prefill calls (0: skip)")
     ap.add_argument("--layers", type=int, default=0, help="layer caches cycled (0: 2 x L2 rule)")
     ap.add_argument("--e2e-steps", type=int, default=256)
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle timing")
@@ -339,6 +397,8 @@ def main():
         ap.error("--warmup must be >= 3")
 
     world, rank, local = dist_env()
+    if args.workload == "prefill":
+        return main_prefill(args)
     w = WORKLOADS[args.workload]
     lens = ref_lens_for(w)
     config = {"workload": w["desc"], "batch": w["B"], "heads": w["H"], "head_dim": w["d"], "n": w["n"],
@@ -378,6 +438,7 @@ def main():
             v, threads, sample = oracle_sample(w, lens, args.cpu_budget)
             cpu = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample}
         value = res["tok_sum"] / res["el_max"]
+        prefill = run_prefill(args.prefill_iters, 3) if (args.prefill_iters > 0 and world == 1) else None
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": res["K"],
             "warmup": args.warmup, "ms_per_step": 1e3 * res["el_max"] / res["K"], "higher_is_better": True,
@@ -400,11 +461,30 @@ def main():
                     "steps": res["K_e2e"]},
             "gpu_launches": res["launches"],
             "cpu_baseline": cpu,
+            "prefill": prefill,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+    return 0
+
+
+def main_prefill(args):
+    """--workload prefill: the teacher-forced form on its own JSON line."""
+    import torch
+    world, rank, local = dist_env()
+    if rank != 0:
+        return 0
+    torch.cuda.set_device(local)
+    r = run_prefill(max(1, args.steps), max(3, args.warmup))
+    line = {"metric": "R-SWA masked prefill TFLOP/s (algorithmic, visible pairs only)", "value": r["tflops"],
+            "unit": "TFLOP/s", "n_gpus": 1, "steps": r["iters"], "warmup": max(3, args.warmup),
+            "ms_per_step": r["ms_per_call"], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": r["workload"], "l2": "inputs 252 MB, larger than L2"},
+            "roofline": r["roofline"], "gpu_launches": r["iters"]}
+    print(json.dumps(line), flush=True)
     return 0
 
 

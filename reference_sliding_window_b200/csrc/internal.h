@@ -118,5 +118,7 @@ struct MaskedParams {
 void set_last_error(const char* prefix, const char* msg);
 
 cudaError_t launch_masked_forward_simt(const MaskedParams& p, int elem, cudaStream_t stream);
+// bf16, head dim 128: tcgen05 tensor-core kernel.
+cudaError_t launch_masked_forward_tc(const MaskedParams& p, cudaStream_t stream);
 
 }  // namespace rswa

@@ -1,0 +1,532 @@
+// Teacher-forced R-SWA attention on the 5th-generation tensor cores
+// (tcgen05 + TMEM), bf16 inputs, head dim 128, float32 accumulation.
+//
+// Operation ("Unlimited OCR Works：一篇读懂 R-SWA 如何把长文档 OCR 从 for-loop 推向
+// one-shot", 方法展开 §3, Eq.(1)-(4), in the packed form used for training on
+// 32K sequences, 实验与证据 §1): O = softmax(Q K^T * scale + M) V per head, where
+// the query at 0-based row i sees key j iff
+//   j <= i  and  (i < L_m  or  j < L_m  or  j > i - n).
+//
+// Design (B200):
+// * One CTA per (128-query tile, head); the grid is ordered heaviest tile
+//   first so that the hardware block scheduler approximates longest-job-first.
+// * The key tiles a query tile needs are the reference tiles [0, ceil(L_m/128))
+//   plus the 2-3 tiles of its causal band; every other tile is fully masked
+//   and skipped.  Only tiles that are not fully visible are masked per element.
+// * Warp 0 lane 0 loads Q once and streams K/V tiles with TMA (128B-swizzled
+//   boxes of 128 rows x 64 columns) into a 2-stage ring.  Warp 1 owns the
+//   tensor memory (512 columns: S double-buffered, O) and one lane issues the
+//   MMAs: S_j = Q K_j^T into TMEM, then O += P_{j-1} V_{j-1}, so the QK^T of
+//   tile j overlaps the softmax of tile j-1.  Warps 2-5 (one thread per query
+//   row) read S with tcgen05.ld, apply the mask and an online softmax in base 2,
+//   write P (bf16, swizzled) to shared memory, and rescale O in TMEM only when
+//   the row maximum grew by more than 2^8 since the last rescale (the stale
+//   maximum keeps every exponent <= 2^8, exact in float32).
+// * Every wait is bounded; on a timeout the kernel marks its rows with NaN,
+//   drains its copies and MMAs, frees its tensor memory and returns.
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+// Exponentials per 8 columns of an unmasked tile evaluated on the FMA pipe
+// (the rest use the XU pipe's ex2).
+#ifndef RSWA_EMU_EIGHTHS
+#define RSWA_EMU_EIGHTHS 3
+#endif
+
+namespace rswa {
+namespace tc {
+
+constexpr int kTile = 128;     // query and key tile
+constexpr int kD = 128;        // head dim
+constexpr int kBox = 64;       // columns per 128B-swizzled box (bf16)
+constexpr int kBoxBytes = kTile * kBox * 2;      // 16 KB
+constexpr int kTileBytes = 2 * kBoxBytes;        // 32 KB: 128 rows x 128 cols
+constexpr int kKV = 2;                           // K/V ring stages
+constexpr int kThreads = 192;                    // producer, MMA, 4 softmax warps
+constexpr int kTmemCols = 512;
+constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
+
+// Shared memory map (offsets from a 1024-byte aligned base).
+constexpr int kSmQ = 0;
+constexpr int kSmK = kSmQ + kTileBytes;
+constexpr int kSmV = kSmK + kKV * kTileBytes;
+constexpr int kSmP = kSmV + kKV * kTileBytes;
+constexpr int kSmBar = kSmP + kTileBytes;        // barriers follow the tiles
+constexpr int kSmBytes = kSmBar + 256 + 1024;    // + slack for 1024-byte alignment
+
+// Instruction descriptor of tcgen05.mma kind::f16: bf16 A and B, float32 D,
+// M = 128, N = 128, A K-major, B K-major (QK^T) or N-major (PV).
+constexpr uint32_t kIdescBase = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kTile >> 3) << 17) |
+                                ((uint32_t)(kTile >> 4) << 24);
+constexpr uint32_t kIdescQK = kIdescBase;
+constexpr uint32_t kIdescPV = kIdescBase | (1u << 16);
+
+// Shared-memory matrix descriptor, 128B swizzle, sm_100 version bit.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int c0, int c1, int c2,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
+      ::"r"(dst), "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}"
+      ::"r"(tmem_d), "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(0), "r"(0), "r"(0), "r"(0)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// 32 consecutive TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+      ::"r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+        "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+        "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+        "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+        "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+        "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+        "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+        "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+        "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+        "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+        "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// 2^x on the FMA pipe, to take part of the exponentials off the XU pipe:
+// n = round(x) with the 1.5*2^23 shifter (Cody-Waite style range reduction),
+// f = x - n in [-1/2, 1/2], 2^f by a cubic, then n is added to the exponent
+// field.  The cubic is the relative least-squares fit of 2^f at Chebyshev
+// nodes computed by fit_exp2.py (relative error <= 7.8e-5, far below the
+// bf16 rounding of P).  For x >= -126 only; callers use it on unmasked tiles.
+__device__ __forceinline__ float exp2_fma(float x) {
+  constexpr float kC0 = 0.99992895f, kC1 = 0.6932762f, kC2 = 0.24260405f, kC3 = 0.055088684f;
+  constexpr float kShift = 12582912.f;  // 1.5 * 2^23
+  x = fmaxf(x, -126.f);
+  const float y = x + kShift;
+  const float f = x - (y - kShift);
+  const float p = fmaf(fmaf(fmaf(kC3, f, kC2), f, kC1), f, kC0);
+  return __int_as_float(__float_as_int(p) + ((__float_as_int(y) - __float_as_int(kShift)) << 23));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+struct TcParams {
+  CUtensorMap tmQ, tmK, tmV;  // 3-D maps {d, H, L} of bf16, 64x1x128 boxes, 128B swizzle
+  __nv_bfloat16* O;
+  int L, L_m, n, H, n_qtiles;
+  float scale_log2;
+};
+
+// Key tiles of query tile qt: [0, A) then [B0, B1] (B0 > A-1 or empty).
+struct TileRange {
+  int A, B0, B1;
+};
+
+__device__ __forceinline__ TileRange tile_range(int q0, int L, int L_m, int n) {
+  const int q_last = min(q0 + kTile, L) - 1;
+  TileRange r;
+  if (q_last < L_m) {  // all prefix rows: causal
+    r.A = q_last / kTile + 1;
+    r.B0 = 1;
+    r.B1 = 0;
+    return r;
+  }
+  r.A = (L_m + kTile - 1) / kTile;
+  const int lo = max(L_m, max(q0, L_m) - n + 1);
+  r.B0 = max(r.A, lo / kTile);
+  r.B1 = q_last / kTile;
+  return r;
+}
+
+__device__ __forceinline__ int tile_count(const TileRange& r) { return r.A + max(0, r.B1 - r.B0 + 1); }
+__device__ __forceinline__ int tile_at(const TileRange& r, int j) { return j < r.A ? j : r.B0 + (j - r.A); }
+
+__global__ void __launch_bounds__(kThreads, 1) masked_tc_kernel(const __grid_constant__ TcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSmBar);
+  // barrier slots
+  const uint32_t b_q = smem_u32(&bars[0]);
+  const uint32_t b_kfull = smem_u32(&bars[1]);   // [kKV]
+  const uint32_t b_vfull = smem_u32(&bars[3]);   // [kKV]
+  const uint32_t b_kvfree = smem_u32(&bars[5]);  // [kKV]
+  const uint32_t b_sfull = smem_u32(&bars[7]);   // [2]
+  const uint32_t b_sfree = smem_u32(&bars[9]);   // [2]
+  const uint32_t b_pfull = smem_u32(&bars[11]);
+  const uint32_t b_odone = smem_u32(&bars[12]);
+  const uint32_t b_final = smem_u32(&bars[13]);
+  volatile uint32_t* s_tmem = reinterpret_cast<volatile uint32_t*>(&bars[14]);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(&bars[15]);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // heaviest tiles first: the tiles holding output rows, then prefix tiles
+  // from the largest down
+  const int h = blockIdx.x % p.H;
+  const int rank = blockIdx.x / p.H;
+  const int t_s = p.L_m / kTile;  // tiles made only of prefix rows
+  const int qt = rank < p.n_qtiles - t_s ? t_s + rank : t_s - 1 - (rank - (p.n_qtiles - t_s));
+  const int q0 = qt * kTile;
+  const TileRange tr = tile_range(q0, p.L, p.L_m, p.n);
+  const int nt = tile_count(tr);
+
+  if (threadIdx.x == 0) {
+    mbar_init(b_q, 1);
+    for (int s = 0; s < kKV; ++s) {
+      mbar_init(b_kfull + 8 * s, 1);
+      mbar_init(b_vfull + 8 * s, 1);
+      mbar_init(b_kvfree + 8 * s, 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(b_sfull + 8 * s, 1);
+      mbar_init(b_sfree + 8 * s, 128);
+    }
+    mbar_init(b_pfull, 128);
+    mbar_init(b_odone, 1);
+    mbar_init(b_final, 1);
+    *s_abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {  // one warp allocates the tensor memory
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32((const void*)s_tmem)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(b_q, kTileBytes);
+      tma_load_3d(sbase + kSmQ, &p.tmQ, 0, h, q0, b_q);
+      tma_load_3d(sbase + kSmQ + kBoxBytes, &p.tmQ, kBox, h, q0, b_q);
+      int issued = 0;
+      for (int j = 0; j < nt; ++j) {
+        const int s = j % kKV;
+        if (*s_abort || !mbar_wait_bounded(b_kvfree + 8 * s, ((j / kKV) & 1) ^ 1)) {
+          *s_abort = 1;
+          break;
+        }
+        const int k0 = tile_at(tr, j) * kTile;
+        mbar_arrive_expect_tx(b_kfull + 8 * s, kTileBytes);
+        tma_load_3d(sbase + kSmK + s * kTileBytes, &p.tmK, 0, h, k0, b_kfull + 8 * s);
+        tma_load_3d(sbase + kSmK + s * kTileBytes + kBoxBytes, &p.tmK, kBox, h, k0, b_kfull + 8 * s);
+        mbar_arrive_expect_tx(b_vfull + 8 * s, kTileBytes);
+        tma_load_3d(sbase + kSmV + s * kTileBytes, &p.tmV, 0, h, k0, b_vfull + 8 * s);
+        tma_load_3d(sbase + kSmV + s * kTileBytes + kBoxBytes, &p.tmV, kBox, h, k0, b_vfull + 8 * s);
+        issued = j + 1;
+      }
+      // drain: every issued copy has landed before the CTA may exit
+      mbar_wait_bounded(b_q, 0);
+      for (int j = max(0, issued - kKV); j < issued; ++j) {
+        mbar_wait_bounded(b_kfull + 8 * (j % kKV), (j / kKV) & 1);
+        mbar_wait_bounded(b_vfull + 8 * (j % kKV), (j / kKV) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      bool ok = mbar_wait_bounded(b_q, 0);
+      const uint32_t aQ = sbase + kSmQ, aP = sbase + kSmP;
+      for (int j = 0; j <= nt && ok; ++j) {
+        if (j < nt) {  // S_j = Q K_j^T
+          const int s = j % kKV, sb = j & 1;
+          ok = !*s_abort && mbar_wait_bounded(b_kfull + 8 * s, (j / kKV) & 1) &&
+               mbar_wait_bounded(b_sfree + 8 * sb, ((j >> 1) & 1) ^ 1);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t aK = sbase + kSmK + s * kTileBytes;
+          const uint32_t dS = tmem + (sb ? kColS1 : kColS0);
+#pragma unroll
+          for (int kk = 0; kk < kD / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
+            mma_bf16(dS, smem_desc(aQ + off, 16, 1024), smem_desc(aK + off, 16, 1024), kIdescQK, kk > 0);
+          }
+          mma_commit(b_sfull + 8 * sb);
+        }
+        if (j >= 1) {  // O += P_{j-1} V_{j-1}
+          const int jp = j - 1, s = jp % kKV;
+          ok = !*s_abort && mbar_wait_bounded(b_pfull, jp & 1) && mbar_wait_bounded(b_vfull + 8 * s, (jp / kKV) & 1);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t aV = sbase + kSmV + s * kTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk) {
+            const uint32_t offP = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
+            mma_bf16(tmem + kColO, smem_desc(aP + offP, 16, 1024), smem_desc(aV + kk * 2048, kBoxBytes, 1024),
+                     kIdescPV, (jp > 0 || kk > 0));
+          }
+          mma_commit(b_odone);
+          mma_commit(b_kvfree + 8 * s);
+        }
+      }
+      if (!ok) *s_abort = 1;
+      // every MMA issued by this thread has completed before TMEM is freed
+      mma_commit(b_final);
+      mbar_wait_bounded(b_final, 0);
+    }
+  } else {
+    // ---------------------------------------------------------- softmax
+    const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
+    const int r = quarter * 32 + lane;
+    const int i = q0 + r;  // query row
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    float m_ref = -INFINITY, l_sum = 0.f;
+    bool ok = true;
+    uint8_t* Prow = smem + kSmP + r * 128;  // row r of both P boxes
+    for (int j = 0; j < nt; ++j) {
+      const int sb = j & 1;
+      if (*s_abort || !mbar_wait_bounded(b_sfull + 8 * sb, (j >> 1) & 1)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float s[kTile];
+#pragma unroll
+      for (int c = 0; c < kTile; c += 32) tmem_ld32(lane_base + (sb ? kColS1 : kColS0) + c, s + c);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(b_sfree + 8 * sb);
+
+      // mask (partial tiles only), row maximum on the raw scores
+      const int k0 = tile_at(tr, j) * kTile;
+      const bool full = (k0 + kTile - 1 < p.L_m) && (q0 >= p.L_m || k0 + kTile - 1 <= q0);
+      float mt = -INFINITY;
+      if (full) {
+#pragma unroll
+        for (int c = 0; c < kTile; ++c) mt = fmaxf(mt, s[c]);
+      } else {
+        // the row's visible columns are [0, ra) and [wb, we]: the reference
+        // keys (causal for a prefix row) and the output window
+        int ra, wb, we;
+        if (i < p.L_m) {
+          ra = i + 1 - k0;
+          wb = 1;
+          we = 0;
+        } else {
+          ra = p.L_m - k0;
+          wb = max(p.L_m, i - p.n + 1) - k0;
+          we = i - k0;
+        }
+#pragma unroll
+        for (int c = 0; c < kTile; ++c) {
+          const bool vis = c < ra || (c >= wb && c <= we);
+          s[c] = vis ? s[c] : -INFINITY;
+          mt = fmaxf(mt, s[c]);
+        }
+      }
+      // lazy rescale: only when the max (log2 units) grew by more than 8
+      const float mt_s = mt * p.scale_log2;
+      const bool grow = mt_s > m_ref + 8.f;
+      const float m_new = grow ? mt_s : m_ref;
+      const float corr = grow ? ex2(m_ref - m_new) : 1.f;  // 0 when m_ref was -inf
+      const float msub = (m_new == -INFINITY) ? 0.f : m_new;
+      // exponentials, packed to bf16 pairs as they are made (64 live registers
+      // instead of 128); RSWA_EMU_EIGHTHS of every 8 columns of unmasked tiles
+      // on the FMA pipe
+      float lt = 0.f;
+      uint32_t pk[kTile / 2];
+      if (full) {
+#pragma unroll
+        for (int c = 0; c < kTile; c += 2) {
+          const float x0 = fmaf(s[c], p.scale_log2, -msub);
+          const float x1 = fmaf(s[c + 1], p.scale_log2, -msub);
+          const float p0 = ((c & 7) < RSWA_EMU_EIGHTHS) ? exp2_fma(x0) : ex2(x0);  // compile-time choice
+          const float p1 = (((c + 1) & 7) < RSWA_EMU_EIGHTHS) ? exp2_fma(x1) : ex2(x1);
+          lt += p0 + p1;
+          pk[c / 2] = pack_bf16x2(p0, p1);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < kTile; c += 2) {
+          const float p0 = ex2(fmaf(s[c], p.scale_log2, -msub));  // masked: -inf -> 0
+          const float p1 = ex2(fmaf(s[c + 1], p.scale_log2, -msub));
+          lt += p0 + p1;
+          pk[c / 2] = pack_bf16x2(p0, p1);
+        }
+      }
+      // P buffer and O are free once PV_{j-1} has completed
+      if (j >= 1) {
+        if (!mbar_wait_bounded(b_odone, (j - 1) & 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, grow)) {
+#pragma unroll 1
+          for (int c = 0; c < kD; c += 32) {
+            float o[32];
+            tmem_ld32(lane_base + kColO + c, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] *= corr;
+            tmem_st32(lane_base + kColO + c, o);
+          }
+          tmem_wait_st();
+        }
+      }
+      l_sum = l_sum * corr + lt;
+      m_ref = m_new;
+      // P row: 128 bf16 as 16 chunks of 16 bytes, 128B-swizzled per box
+#pragma unroll
+      for (int cc = 0; cc < 16; ++cc) {
+        const uint4 w = make_uint4(pk[cc * 4 + 0], pk[cc * 4 + 1], pk[cc * 4 + 2], pk[cc * 4 + 3]);
+        const int box = cc >> 3, chunk = (cc & 7) ^ (r & 7);
+        *reinterpret_cast<uint4*>(Prow + box * kBoxBytes + chunk * 16) = w;
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // P visible to the tensor core
+      tc_fence_before();
+      mbar_arrive(b_pfull);
+    }
+    // epilogue: O / l to global memory
+    if (ok && nt > 0 && !mbar_wait_bounded(b_odone, (nt - 1) & 1)) ok = false;
+    tc_fence_after();
+    if (!ok) *s_abort = 1;
+    __nv_bfloat16* orow = p.O + ((size_t)i * p.H + h) * kD;
+    const float inv = ok ? 1.f / l_sum : __int_as_float(0x7fc00000);
+#pragma unroll 1
+    for (int c = 0; c < kD; c += 32) {
+      float o[32];
+      tmem_ld32(lane_base + kColO + c, o);
+      tmem_wait_ld();
+      if (i < p.L) {
+#pragma unroll
+        for (int e = 0; e < 32; e += 8) {
+          uint4 w;
+          w.x = pack_bf16x2(o[e] * inv, o[e + 1] * inv);
+          w.y = pack_bf16x2(o[e + 2] * inv, o[e + 3] * inv);
+          w.z = pack_bf16x2(o[e + 4] * inv, o[e + 5] * inv);
+          w.w = pack_bf16x2(o[e + 6] * inv, o[e + 7] * inv);
+          *reinterpret_cast<uint4*>(orow + c + e) = w;
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                              : "memory");
+}
+
+// ---------------------------------------------------------------- host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+static bool make_map(CUtensorMap* m, const void* base, int L, int H) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)L};
+  const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)H * kD * 2};
+  const cuuint32_t box[3] = {(cuuint32_t)kBox, 1, (cuuint32_t)kTile};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace tc
+
+cudaError_t launch_masked_forward_tc(const MaskedParams& mp, cudaStream_t stream) {
+  using namespace tc;
+  TcParams p;
+  if (!make_map(&p.tmQ, mp.Q, mp.L, mp.H) || !make_map(&p.tmK, mp.K, mp.L, mp.H) ||
+      !make_map(&p.tmV, mp.V, mp.L, mp.H))
+    return cudaErrorInvalidValue;
+  p.O = static_cast<__nv_bfloat16*>(mp.O);
+  p.L = mp.L;
+  p.L_m = mp.L_m;
+  p.n = mp.n;
+  p.H = mp.H;
+  p.n_qtiles = (mp.L + kTile - 1) / kTile;
+  p.scale_log2 = mp.scale_log2;
+  static bool configured[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(masked_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmBytes);
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  masked_tc_kernel<<<p.n_qtiles * p.H, kThreads, kSmBytes, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace rswa
