@@ -17,11 +17,14 @@
 //   boxes of 128 rows x 64 columns) into a 2-stage ring.  Warp 1 owns the
 //   tensor memory (512 columns: S double-buffered, O) and one lane issues the
 //   MMAs: S_j = Q K_j^T into TMEM, then O += P_{j-1} V_{j-1}, so the QK^T of
-//   tile j overlaps the softmax of tile j-1.  Warps 2-5 (one thread per query
-//   row) read S with tcgen05.ld, apply the mask and an online softmax in base 2,
-//   write P (bf16, swizzled) to shared memory, and rescale O in TMEM only when
-//   the row maximum grew by more than 2^8 since the last rescale (the stale
-//   maximum keeps every exponent <= 2^8, exact in float32).
+//   tile j overlaps the softmax of tile j-1.
+// * Warps 2.. run the softmax, kSplit threads per query row: warps w, w+4, ...
+//   read the same TMEM lanes, each taking 128/kSplit columns.  The parts of a
+//   row exchange their maxima through shared memory (one named barrier per
+//   tile), form p = 2^(s*scale*log2e - m), write their part of P (bf16,
+//   128B-swizzled) for the PV MMA, and rescale their part of O in TMEM
+//   only when the row maximum grew by more than 2^8 since the last rescale
+//   (the stale maximum keeps every exponent <= 2^8, exact in float32).
 // * Every wait is bounded; on a timeout the kernel marks its rows with NaN,
 //   drains its copies and MMAs, frees its tensor memory and returns.
 
@@ -38,7 +41,7 @@
 // Exponentials per 8 columns of an unmasked tile evaluated on the FMA pipe
 // (the rest use the XU pipe's ex2).
 #ifndef RSWA_EMU_EIGHTHS
-#define RSWA_EMU_EIGHTHS 3
+#define RSWA_EMU_EIGHTHS 0  // measured on B200: enabling it slowed the kernel down
 #endif
 
 namespace rswa {
@@ -46,11 +49,17 @@ namespace tc {
 
 constexpr int kTile = 128;     // query and key tile
 constexpr int kD = 128;        // head dim
+#ifndef RSWA_TC_SPLIT
+#define RSWA_TC_SPLIT 2
+#endif
+constexpr int kSplit = RSWA_TC_SPLIT;  // softmax threads per query row
+constexpr int kHalf = 128 / kSplit;    // columns per softmax thread
 constexpr int kBox = 64;       // columns per 128B-swizzled box (bf16)
 constexpr int kBoxBytes = kTile * kBox * 2;      // 16 KB
 constexpr int kTileBytes = 2 * kBoxBytes;        // 32 KB: 128 rows x 128 cols
 constexpr int kKV = 2;                           // K/V ring stages
-constexpr int kThreads = 192;                    // producer, MMA, 4 softmax warps
+constexpr int kSoftmaxThreads = 128 * kSplit;    // warps 2 .. 2 + 4*kSplit - 1
+constexpr int kThreads = 64 + kSoftmaxThreads;   // producer, MMA, softmax
 constexpr int kTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
 
@@ -59,7 +68,8 @@ constexpr int kSmQ = 0;
 constexpr int kSmK = kSmQ + kTileBytes;
 constexpr int kSmV = kSmK + kKV * kTileBytes;
 constexpr int kSmP = kSmV + kKV * kTileBytes;
-constexpr int kSmBar = kSmP + kTileBytes;        // barriers follow the tiles
+constexpr int kSmRed = kSmP + kTileBytes;        // float rmax[2][kSplit][128], lsum[kSplit][128]
+constexpr int kSmBar = kSmRed + (2 * kSplit * kTile + kSplit * kTile) * 4;
 constexpr int kSmBytes = kSmBar + 256 + 1024;    // + slack for 1024-byte alignment
 
 // Instruction descriptor of tcgen05.mma kind::f16: bf16 A and B, float32 D,
@@ -135,6 +145,32 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
       : "memory");
 }
 
+// 16 consecutive TMEM columns of this thread's lane (load and store).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+      ::"r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+        "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+        "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+        "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+        "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+        "r"(__float_as_uint(v[15]))
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -173,7 +209,7 @@ struct TcParams {
   float scale_log2;
 };
 
-// Key tiles of query tile qt: [0, A) then [B0, B1] (B0 > A-1 or empty).
+// Key tiles of query tile at q0: [0, A) then [B0, B1] (B0 > A-1 or empty).
 struct TileRange {
   int A, B0, B1;
 };
@@ -197,23 +233,62 @@ __device__ __forceinline__ TileRange tile_range(int q0, int L, int L_m, int n) {
 __device__ __forceinline__ int tile_count(const TileRange& r) { return r.A + max(0, r.B1 - r.B0 + 1); }
 __device__ __forceinline__ int tile_at(const TileRange& r, int j) { return j < r.A ? j : r.B0 + (j - r.A); }
 
+// Barrier slots (8 bytes each).
+enum : int {
+  kBarQ = 0, kBarKFull = 1, kBarVFull = 3, kBarKVFree = 5, kBarSFull = 7, kBarSFree = 9,
+  kBarPFull = 11, kBarODone = 12, kBarFinal = 13, kSlotTmem = 14, kSlotAbort = 15
+};
+
+// One thread's half row of an S tile (64 columns starting at col0):
+// maximum of the visible scores.  FULL: every column visible; otherwise the
+// row's visible columns are [0, ra) and [wb, we] (the reference keys, causal
+// for a prefix row, and the output window).
+template <bool FULL>
+__device__ __forceinline__ float half_max(const float* s, int col0, int ra, int wb, int we) {
+  float m8[8];  // independent chains: 8 steps deep instead of 64
+#pragma unroll
+  for (int k = 0; k < 8; ++k) m8[k] = -INFINITY;
+#pragma unroll
+  for (int e = 0; e < kHalf; ++e) {
+    const int c = col0 + e;
+    m8[e & 7] = fmaxf(m8[e & 7], (FULL || c < ra || (c >= wb && c <= we)) ? s[e] : -INFINITY);
+  }
+  return fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+}
+
+// Exponentials of the half row, packed to bf16 pairs; returns their sum.
+template <bool FULL>
+__device__ __forceinline__ float half_exp(const float* s, int col0, int ra, int wb, int we, float sl2, float msub,
+                                          uint32_t* pk) {
+  float l4[4] = {0.f, 0.f, 0.f, 0.f};  // independent sums
+#pragma unroll
+  for (int e = 0; e < kHalf; e += 2) {
+    const int c = col0 + e;
+    float x0 = fmaf(s[e], sl2, -msub), x1 = fmaf(s[e + 1], sl2, -msub);
+    if (!FULL) {  // masked columns: exponent -inf gives exactly 0
+      x0 = (c < ra || (c >= wb && c <= we)) ? x0 : -INFINITY;
+      x1 = (c + 1 < ra || (c + 1 >= wb && c + 1 <= we)) ? x1 : -INFINITY;
+    }
+    // the column pattern choosing the FMA-pipe exponential is a compile-time constant
+    const float p0 = (FULL && (e & 7) < RSWA_EMU_EIGHTHS) ? exp2_fma(x0) : ex2(x0);
+    const float p1 = (FULL && ((e + 1) & 7) < RSWA_EMU_EIGHTHS) ? exp2_fma(x1) : ex2(x1);
+    l4[(e >> 1) & 3] += p0 + p1;
+    pk[e / 2] = pack_bf16x2(p0, p1);
+  }
+  return (l4[0] + l4[1]) + (l4[2] + l4[3]);
+}
+
 __global__ void __launch_bounds__(kThreads, 1) masked_tc_kernel(const __grid_constant__ TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSmBar);
-  // barrier slots
-  const uint32_t b_q = smem_u32(&bars[0]);
-  const uint32_t b_kfull = smem_u32(&bars[1]);   // [kKV]
-  const uint32_t b_vfull = smem_u32(&bars[3]);   // [kKV]
-  const uint32_t b_kvfree = smem_u32(&bars[5]);  // [kKV]
-  const uint32_t b_sfull = smem_u32(&bars[7]);   // [2]
-  const uint32_t b_sfree = smem_u32(&bars[9]);   // [2]
-  const uint32_t b_pfull = smem_u32(&bars[11]);
-  const uint32_t b_odone = smem_u32(&bars[12]);
-  const uint32_t b_final = smem_u32(&bars[13]);
-  volatile uint32_t* s_tmem = reinterpret_cast<volatile uint32_t*>(&bars[14]);
-  volatile int* s_abort = reinterpret_cast<volatile int*>(&bars[15]);
+  const uint32_t bar0 = smem_u32(bars);
+  auto B = [&](int slot) { return bar0 + 8u * slot; };
+  volatile uint32_t* s_tmem = reinterpret_cast<volatile uint32_t*>(&bars[kSlotTmem]);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(&bars[kSlotAbort]);
+  float* rmax = reinterpret_cast<float*>(smem + kSmRed);  // [parity][part][row]
+  float* lsum = rmax + 2 * kSplit * kTile;                 // [part][row]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -228,19 +303,19 @@ __global__ void __launch_bounds__(kThreads, 1) masked_tc_kernel(const __grid_con
   const int nt = tile_count(tr);
 
   if (threadIdx.x == 0) {
-    mbar_init(b_q, 1);
+    mbar_init(B(kBarQ), 1);
     for (int s = 0; s < kKV; ++s) {
-      mbar_init(b_kfull + 8 * s, 1);
-      mbar_init(b_vfull + 8 * s, 1);
-      mbar_init(b_kvfree + 8 * s, 1);
+      mbar_init(B(kBarKFull + s), 1);
+      mbar_init(B(kBarVFull + s), 1);
+      mbar_init(B(kBarKVFree + s), 1);
     }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(b_sfull + 8 * s, 1);
-      mbar_init(b_sfree + 8 * s, 128);
+      mbar_init(B(kBarSFull + s), 1);
+      mbar_init(B(kBarSFree + s), kSoftmaxThreads);
     }
-    mbar_init(b_pfull, 128);
-    mbar_init(b_odone, 1);
-    mbar_init(b_final, 1);
+    mbar_init(B(kBarPFull), kSoftmaxThreads);
+    mbar_init(B(kBarODone), 1);
+    mbar_init(B(kBarFinal), 1);
     *s_abort = 0;
     fence_barrier_init();
   }
@@ -258,42 +333,42 @@ __global__ void __launch_bounds__(kThreads, 1) masked_tc_kernel(const __grid_con
   if (warp == 0) {
     // ---------------------------------------------------------- producer
     if (lane == 0) {
-      mbar_arrive_expect_tx(b_q, kTileBytes);
-      tma_load_3d(sbase + kSmQ, &p.tmQ, 0, h, q0, b_q);
-      tma_load_3d(sbase + kSmQ + kBoxBytes, &p.tmQ, kBox, h, q0, b_q);
+      mbar_arrive_expect_tx(B(kBarQ), kTileBytes);
+      tma_load_3d(sbase + kSmQ, &p.tmQ, 0, h, q0, B(kBarQ));
+      tma_load_3d(sbase + kSmQ + kBoxBytes, &p.tmQ, kBox, h, q0, B(kBarQ));
       int issued = 0;
       for (int j = 0; j < nt; ++j) {
         const int s = j % kKV;
-        if (*s_abort || !mbar_wait_bounded(b_kvfree + 8 * s, ((j / kKV) & 1) ^ 1)) {
+        if (*s_abort || !mbar_wait_bounded(B(kBarKVFree + s), ((j / kKV) & 1) ^ 1)) {
           *s_abort = 1;
           break;
         }
         const int k0 = tile_at(tr, j) * kTile;
-        mbar_arrive_expect_tx(b_kfull + 8 * s, kTileBytes);
-        tma_load_3d(sbase + kSmK + s * kTileBytes, &p.tmK, 0, h, k0, b_kfull + 8 * s);
-        tma_load_3d(sbase + kSmK + s * kTileBytes + kBoxBytes, &p.tmK, kBox, h, k0, b_kfull + 8 * s);
-        mbar_arrive_expect_tx(b_vfull + 8 * s, kTileBytes);
-        tma_load_3d(sbase + kSmV + s * kTileBytes, &p.tmV, 0, h, k0, b_vfull + 8 * s);
-        tma_load_3d(sbase + kSmV + s * kTileBytes + kBoxBytes, &p.tmV, kBox, h, k0, b_vfull + 8 * s);
+        mbar_arrive_expect_tx(B(kBarKFull + s), kTileBytes);
+        tma_load_3d(sbase + kSmK + s * kTileBytes, &p.tmK, 0, h, k0, B(kBarKFull + s));
+        tma_load_3d(sbase + kSmK + s * kTileBytes + kBoxBytes, &p.tmK, kBox, h, k0, B(kBarKFull + s));
+        mbar_arrive_expect_tx(B(kBarVFull + s), kTileBytes);
+        tma_load_3d(sbase + kSmV + s * kTileBytes, &p.tmV, 0, h, k0, B(kBarVFull + s));
+        tma_load_3d(sbase + kSmV + s * kTileBytes + kBoxBytes, &p.tmV, kBox, h, k0, B(kBarVFull + s));
         issued = j + 1;
       }
       // drain: every issued copy has landed before the CTA may exit
-      mbar_wait_bounded(b_q, 0);
+      mbar_wait_bounded(B(kBarQ), 0);
       for (int j = max(0, issued - kKV); j < issued; ++j) {
-        mbar_wait_bounded(b_kfull + 8 * (j % kKV), (j / kKV) & 1);
-        mbar_wait_bounded(b_vfull + 8 * (j % kKV), (j / kKV) & 1);
+        mbar_wait_bounded(B(kBarKFull + j % kKV), (j / kKV) & 1);
+        mbar_wait_bounded(B(kBarVFull + j % kKV), (j / kKV) & 1);
       }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      bool ok = mbar_wait_bounded(b_q, 0);
+      bool ok = mbar_wait_bounded(B(kBarQ), 0);
       const uint32_t aQ = sbase + kSmQ, aP = sbase + kSmP;
       for (int j = 0; j <= nt && ok; ++j) {
         if (j < nt) {  // S_j = Q K_j^T
           const int s = j % kKV, sb = j & 1;
-          ok = !*s_abort && mbar_wait_bounded(b_kfull + 8 * s, (j / kKV) & 1) &&
-               mbar_wait_bounded(b_sfree + 8 * sb, ((j >> 1) & 1) ^ 1);
+          ok = !*s_abort && mbar_wait_bounded(B(kBarKFull + s), (j / kKV) & 1) &&
+               mbar_wait_bounded(B(kBarSFree + sb), ((j >> 1) & 1) ^ 1);
           if (!ok) break;
           tc_fence_after();
           const uint32_t aK = sbase + kSmK + s * kTileBytes;
@@ -303,11 +378,12 @@ __global__ void __launch_bounds__(kThreads, 1) masked_tc_kernel(const __grid_con
             const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
             mma_bf16(dS, smem_desc(aQ + off, 16, 1024), smem_desc(aK + off, 16, 1024), kIdescQK, kk > 0);
           }
-          mma_commit(b_sfull + 8 * sb);
+          mma_commit(B(kBarSFull + sb));
         }
         if (j >= 1) {  // O += P_{j-1} V_{j-1}
           const int jp = j - 1, s = jp % kKV;
-          ok = !*s_abort && mbar_wait_bounded(b_pfull, jp & 1) && mbar_wait_bounded(b_vfull + 8 * s, (jp / kKV) & 1);
+          ok = !*s_abort && mbar_wait_bounded(B(kBarPFull), jp & 1) &&
+               mbar_wait_bounded(B(kBarVFull + s), (jp / kKV) & 1);
           if (!ok) break;
           tc_fence_after();
           const uint32_t aV = sbase + kSmV + s * kTileBytes;
@@ -317,138 +393,112 @@ __global__ void __launch_bounds__(kThreads, 1) masked_tc_kernel(const __grid_con
             mma_bf16(tmem + kColO, smem_desc(aP + offP, 16, 1024), smem_desc(aV + kk * 2048, kBoxBytes, 1024),
                      kIdescPV, (jp > 0 || kk > 0));
           }
-          mma_commit(b_odone);
-          mma_commit(b_kvfree + 8 * s);
+          mma_commit(B(kBarODone));
+          mma_commit(B(kBarKVFree + s));
         }
       }
       if (!ok) *s_abort = 1;
       // every MMA issued by this thread has completed before TMEM is freed
-      mma_commit(b_final);
-      mbar_wait_bounded(b_final, 0);
+      mma_commit(B(kBarFinal));
+      mbar_wait_bounded(B(kBarFinal), 0);
     }
   } else {
     // ---------------------------------------------------------- softmax
-    const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
+    const int hf = (warp - 2) >> 2;  // which part of the row: columns kHalf*hf ..
+    const int quarter = warp & 3;    // TMEM lanes 32*quarter .. +31
     const int r = quarter * 32 + lane;
-    const int i = q0 + r;  // query row
+    const int i = q0 + r;            // query row
+    const int col0 = hf * kHalf;
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    // this part of row r of P: box col0/64, first 16-byte chunk (col0 % 64)/8
+    uint8_t* Pbox = smem + kSmP + (col0 / kBox) * kBoxBytes + r * 128;
+    const int chunk0 = (col0 % kBox) / 8;
     float m_ref = -INFINITY, l_sum = 0.f;
     bool ok = true;
-    uint8_t* Prow = smem + kSmP + r * 128;  // row r of both P boxes
     for (int j = 0; j < nt; ++j) {
       const int sb = j & 1;
-      if (*s_abort || !mbar_wait_bounded(b_sfull + 8 * sb, (j >> 1) & 1)) {
-        ok = false;
-        break;
-      }
+      // After a timed-out wait a thread stops waiting but keeps arriving and
+      // joining the named barriers, so no thread of the CTA can be left
+      // waiting on it; its rows are written as NaN.
+      if (ok && (*s_abort || !mbar_wait_bounded(B(kBarSFull + sb), (j >> 1) & 1))) ok = false;
       tc_fence_after();
-      float s[kTile];
+      float s[kHalf];
 #pragma unroll
-      for (int c = 0; c < kTile; c += 32) tmem_ld32(lane_base + (sb ? kColS1 : kColS0) + c, s + c);
+      for (int c = 0; c < kHalf; c += 32) tmem_ld32(lane_base + (sb ? kColS1 : kColS0) + col0 + c, s + c);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(b_sfree + 8 * sb);
+      mbar_arrive(B(kBarSFree + sb));
 
-      // mask (partial tiles only), row maximum on the raw scores
       const int k0 = tile_at(tr, j) * kTile;
       const bool full = (k0 + kTile - 1 < p.L_m) && (q0 >= p.L_m || k0 + kTile - 1 <= q0);
-      float mt = -INFINITY;
-      if (full) {
-#pragma unroll
-        for (int c = 0; c < kTile; ++c) mt = fmaxf(mt, s[c]);
-      } else {
-        // the row's visible columns are [0, ra) and [wb, we]: the reference
-        // keys (causal for a prefix row) and the output window
-        int ra, wb, we;
+      int ra = kTile, wb = 1, we = 0;
+      if (!full) {
         if (i < p.L_m) {
           ra = i + 1 - k0;
-          wb = 1;
-          we = 0;
         } else {
           ra = p.L_m - k0;
           wb = max(p.L_m, i - p.n + 1) - k0;
           we = i - k0;
         }
-#pragma unroll
-        for (int c = 0; c < kTile; ++c) {
-          const bool vis = c < ra || (c >= wb && c <= we);
-          s[c] = vis ? s[c] : -INFINITY;
-          mt = fmaxf(mt, s[c]);
-        }
       }
+      // row maximum: this half, then the other half's through shared memory
+      const float mh = full ? half_max<true>(s, col0, ra, wb, we) : half_max<false>(s, col0, ra, wb, we);
+      rmax[(sb * kSplit + hf) * kTile + r] = mh;
+      named_barrier_sync(1, kSoftmaxThreads);
+      float mt = mh;
+#pragma unroll
+      for (int k = 0; k < kSplit; ++k) mt = fmaxf(mt, rmax[(sb * kSplit + k) * kTile + r]);
       // lazy rescale: only when the max (log2 units) grew by more than 8
       const float mt_s = mt * p.scale_log2;
       const bool grow = mt_s > m_ref + 8.f;
       const float m_new = grow ? mt_s : m_ref;
       const float corr = grow ? ex2(m_ref - m_new) : 1.f;  // 0 when m_ref was -inf
       const float msub = (m_new == -INFINITY) ? 0.f : m_new;
-      // exponentials, packed to bf16 pairs as they are made (64 live registers
-      // instead of 128); RSWA_EMU_EIGHTHS of every 8 columns of unmasked tiles
-      // on the FMA pipe
-      float lt = 0.f;
-      uint32_t pk[kTile / 2];
-      if (full) {
-#pragma unroll
-        for (int c = 0; c < kTile; c += 2) {
-          const float x0 = fmaf(s[c], p.scale_log2, -msub);
-          const float x1 = fmaf(s[c + 1], p.scale_log2, -msub);
-          const float p0 = ((c & 7) < RSWA_EMU_EIGHTHS) ? exp2_fma(x0) : ex2(x0);  // compile-time choice
-          const float p1 = (((c + 1) & 7) < RSWA_EMU_EIGHTHS) ? exp2_fma(x1) : ex2(x1);
-          lt += p0 + p1;
-          pk[c / 2] = pack_bf16x2(p0, p1);
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < kTile; c += 2) {
-          const float p0 = ex2(fmaf(s[c], p.scale_log2, -msub));  // masked: -inf -> 0
-          const float p1 = ex2(fmaf(s[c + 1], p.scale_log2, -msub));
-          lt += p0 + p1;
-          pk[c / 2] = pack_bf16x2(p0, p1);
-        }
-      }
+      uint32_t pk[kHalf / 2];
+      const float lt = full ? half_exp<true>(s, col0, ra, wb, we, p.scale_log2, msub, pk)
+                            : half_exp<false>(s, col0, ra, wb, we, p.scale_log2, msub, pk);
       // P buffer and O are free once PV_{j-1} has completed
-      if (j >= 1) {
-        if (!mbar_wait_bounded(b_odone, (j - 1) & 1)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, grow)) {
-#pragma unroll 1
-          for (int c = 0; c < kD; c += 32) {
-            float o[32];
-            tmem_ld32(lane_base + kColO + c, o);
-            tmem_wait_ld();
+      if (j >= 1 && ok && !mbar_wait_bounded(B(kBarODone), (j - 1) & 1)) ok = false;
+      tc_fence_after();
+      // this part of the P row: kHalf bf16 in 16-byte chunks, 128B-swizzled
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] *= corr;
-            tmem_st32(lane_base + kColO + c, o);
-          }
-          tmem_wait_st();
+      for (int cc = 0; cc < kHalf / 8; ++cc) {
+        const uint4 w = make_uint4(pk[cc * 4 + 0], pk[cc * 4 + 1], pk[cc * 4 + 2], pk[cc * 4 + 3]);
+        *reinterpret_cast<uint4*>(Pbox + (((chunk0 + cc) ^ (r & 7)) * 16)) = w;
+      }
+      if (j >= 1 && __any_sync(0xffffffffu, grow)) {
+#pragma unroll 1
+        for (int c = 0; c < kHalf; c += 16) {
+          float o[16];
+          tmem_ld16(lane_base + kColO + col0 + c, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) o[e] *= corr;
+          tmem_st16(lane_base + kColO + col0 + c, o);
         }
+        tmem_wait_st();
       }
       l_sum = l_sum * corr + lt;
       m_ref = m_new;
-      // P row: 128 bf16 as 16 chunks of 16 bytes, 128B-swizzled per box
-#pragma unroll
-      for (int cc = 0; cc < 16; ++cc) {
-        const uint4 w = make_uint4(pk[cc * 4 + 0], pk[cc * 4 + 1], pk[cc * 4 + 2], pk[cc * 4 + 3]);
-        const int box = cc >> 3, chunk = (cc & 7) ^ (r & 7);
-        *reinterpret_cast<uint4*>(Prow + box * kBoxBytes + chunk * 16) = w;
-      }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // P visible to the tensor core
       tc_fence_before();
-      mbar_arrive(b_pfull);
+      mbar_arrive(B(kBarPFull));
     }
-    // epilogue: O / l to global memory
-    if (ok && nt > 0 && !mbar_wait_bounded(b_odone, (nt - 1) & 1)) ok = false;
+    // epilogue: O / l to global memory, l summed over both halves
+    if (ok && nt > 0 && (*s_abort || !mbar_wait_bounded(B(kBarODone), (nt - 1) & 1))) ok = false;
     tc_fence_after();
     if (!ok) *s_abort = 1;
-    __nv_bfloat16* orow = p.O + ((size_t)i * p.H + h) * kD;
-    const float inv = ok ? 1.f / l_sum : __int_as_float(0x7fc00000);
+    lsum[hf * kTile + r] = l_sum;
+    named_barrier_sync(1, kSoftmaxThreads);
+    float l_tot = 0.f;
+#pragma unroll
+    for (int k = 0; k < kSplit; ++k) l_tot += lsum[k * kTile + r];
+    const float inv = (ok && !*s_abort) ? 1.f / l_tot : __int_as_float(0x7fc00000);
+    __nv_bfloat16* orow = p.O + ((size_t)i * p.H + h) * kD + col0;
 #pragma unroll 1
-    for (int c = 0; c < kD; c += 32) {
+    for (int c = 0; c < kHalf; c += 32) {
       float o[32];
-      tmem_ld32(lane_base + kColO + c, o);
+      tmem_ld32(lane_base + kColO + col0 + c, o);
       tmem_wait_ld();
       if (i < p.L) {
 #pragma unroll
