@@ -228,6 +228,18 @@ def reduce_max_sum(elapsed_s: float, units: float, backend_device=None):
     return float(t.item()), float(u.item())
 
 
+def replica_seed(base: int, layer: int, rank: int) -> int:
+    """Seed of one rank's inputs: every rank runs its own replica of the
+    workload on different data (no rank shares a tensor with another)."""
+    return base + layer + 7919 * rank
+
+
+def whole_job_rate(units_sum: float, elapsed_max_s: float) -> float:
+    """Whole-job throughput: the units every rank processed over the time of
+    the slowest rank."""
+    return units_sum / elapsed_max_s
+
+
 # --------------------------------------------------------------- our arm
 
 def ref_lens_for(w, seed=0):
@@ -264,13 +276,13 @@ def run_ours(args, w, lens):
     layers = []
     for r in range(R):
         a = RSWA(L_m_cap, n, H, d, B, dt, device=dev)
-        Kr = synth.normal((B, H, L_m_cap, d), 1000 + r + 7919 * rank, w["dtype"], "cuda")
-        Vr = synth.normal((B, H, L_m_cap, d), 2000 + r + 7919 * rank, w["dtype"], "cuda")
+        Kr = synth.normal((B, H, L_m_cap, d), replica_seed(1000, r, rank), w["dtype"], "cuda")
+        Vr = synth.normal((B, H, L_m_cap, d), replica_seed(2000, r, rank), w["dtype"], "cuda")
         a.load_reference(Kr, Vr, lens)
         del Kr, Vr
         layers.append(a)
     P = 16  # distinct per-step inputs, cycled
-    pool = synth.normal((P, R, 3, B, H, d), 3000 + 7919 * rank, w["dtype"], "cuda")
+    pool = synth.normal((P, R, 3, B, H, d), replica_seed(3000, 0, rank), w["dtype"], "cuda")
     out = torch.empty((R, B, H, d), dtype=dt, device=dev)
 
     def step(i):
@@ -437,7 +449,7 @@ def main():
         if world == 1:
             v, threads, sample = oracle_sample(w, lens, args.cpu_budget)
             cpu = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample}
-        value = res["tok_sum"] / res["el_max"]
+        value = whole_job_rate(res["tok_sum"], res["el_max"])
         prefill = run_prefill(args.prefill_iters, 3) if (args.prefill_iters > 0 and world == 1) else None
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": res["K"],
@@ -456,7 +468,7 @@ def main():
                          "algorithmic_bytes_per_launch": res["per_launch"],
                          "avg_launch_us": avg_launch * 1e6, "kernel": "rswa::decode_kernel<bf16,128,append>"},
             "clocks": res["clocks"],
-            "e2e": {"value": res["e2e_tok"] / res["e2e_max"], "unit": "tokens/s",
+            "e2e": {"value": whole_job_rate(res["e2e_tok"], res["e2e_max"]), "unit": "tokens/s",
                     "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"],
                     "steps": res["K_e2e"]},
             "gpu_launches": res["launches"],
