@@ -98,6 +98,11 @@ size_t rswa_workspace_bytes(int L_m_cap, int window_cap, int H, int d, int batch
  *     [0, L_m[b]) hold the reference segment and rows
  *     [L_m[b], L_m[b] + window_cap) the output segment (the n-slot ring in
  *     RSWA mode, outputs in order in FULL mode).
+ *   The caches belong to the handle until rswa_destroy: the caller must not
+ *     write them.  Decode kernels copy reference rows before waiting on the
+ *     preceding kernel of the stream (programmatic dependent launch); this
+ *     is safe because only rswa_load_reference writes those rows and its
+ *     kernel makes its writes visible before it retires.
  *   workspace: rswa_workspace_bytes(...) bytes; zeroed by this call
  *     (stream-ordered).
  *   n: window size (RSWA mode, >= 1).  T_cap: max outputs (FULL mode, >= 1).

@@ -418,6 +418,14 @@ static rswa_status run_decode(rswa_ctx* c, const void* k, const void* v, const v
   const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)c->d);
   p.scale_log2 = sc * 1.4426950408889634f;
   p.timing = g_timing;
+  // Only rswa_load_reference writes the reference rows, and its kernel
+  // fences its writes before retiring, so every later decode may copy them
+  // before its dependency wait.
+#ifdef RSWA_NO_EARLY_COPY
+  p.ref_stable = 0;
+#else
+  p.ref_stable = 1;
+#endif
   const int grid = c->n_ctas;
   RSWA_CUDA(launch_decode(c->dtype == RSWA_BF16 ? kBF16 : kF32, c->d, append, p, grid, c->stream),
             "decode kernel");

@@ -64,6 +64,10 @@ __global__ void __launch_bounds__(256) load_reference_kernel(const __grid_consta
     *reinterpret_cast<uint4*>(kd + i * 16) = *reinterpret_cast<const uint4*>(ks + i * 16);
     *reinterpret_cast<uint4*>(vd + i * 16) = *reinterpret_cast<const uint4*>(vs + i * 16);
   }
+  // Decode kernels launched after this one copy reference rows before their
+  // dependency wait: make this block's writes visible GPU-wide before it
+  // retires.
+  __threadfence();
 }
 
 cudaError_t launch_append(const AppendParams& p, cudaStream_t stream) {

@@ -18,16 +18,22 @@
 //   ring of shared-memory buffers with bulk async copies (cp.async.bulk,
 //   completion on mbarriers).  It needs no device state, so the first copy
 //   is issued right after the plan is read.
-// * Stage g (counted over the launch) goes to consumer warp g % kW and ring
-//   buffer g % kStages.  kStages is a multiple of kW, so a buffer is only
-//   ever consumed by one warp, which waits on it only after consuming its
-//   previous phase: every mbarrier parity wait is unambiguous.
-// * A consumer warp reads a stage with 16-byte shared loads (one row = LPR
-//   lanes), forms LPR partial dot products per lane and reduces them with a
-//   transposed butterfly (LPR-1 shuffles leave every lane one finished
-//   score), then updates a float32 online softmax (base-2 exponent with the
-//   scale folded into q) and its slice of the output.  Rows at or past the
-//   current cache length are masked.
+// * Stage g (32 rows, counted over the launch) goes to consumer warp group
+//   g % kGroups and ring buffer g % kStages; the kSplit warps of a group
+//   each take kWarpRows rows of it.  kStages is a multiple of kGroups, so a
+//   buffer is only ever consumed by one group, whose warps wait on it only
+//   after consuming its previous phase: every mbarrier parity wait is
+//   unambiguous.
+// * A warp's part of a stage is NV = 8 warp-wide 16-byte loads of K (and of
+//   V): 16 rows of bf16 d=128.  The warp reads it from shared memory (one
+//   row = LPR lanes), forms NV partial dot products per lane and reduces
+//   them with a transposed butterfly over NV lanes plus plain shuffles over
+//   the rest of the row's lanes (NV-1 + log2(LPR/NV) shuffles leave every
+//   lane one finished score), then updates a float32 online softmax (base-2
+//   exponent with the scale folded into q) and its slice of the output.
+//   Rows at or past the current cache length are masked.  Splitting stages
+//   over warps keeps the serial work of one warp short (at small cache
+//   sizes the launch is latency-bound) while the copies stay 8 KB each.
 // * Warps merge per item in shared memory.  Items of a shared slab leave a
 //   partial (m, l, o); at the end of its span a CTA takes one acq_rel ticket
 //   per such item and the last CTA of a slab merges its partials with the
@@ -50,10 +56,16 @@
 
 namespace rswa {
 
-constexpr int kStageRows = 32;
 constexpr int kStageBudget = 192 * 1024;
 constexpr long long kPrefetchBytes = 256 * 1024;  // per CTA and per K/V tensor
 constexpr int kPrefetchChunk = 32 * 1024;
+// Items per CTA whose descriptor, reference length and (scaled) query are
+// staged in shared memory by the prologue; later items of a longer span
+// read them from global memory when they start.
+constexpr int kPreItems = 8;
+// Items a CTA processes together: the warps run their stages of both before
+// one barrier, so a span that crosses a slab boundary costs one round.
+constexpr int kBatch = 2;
 
 template <typename T, int D>
 struct DecTraits {
@@ -61,18 +73,28 @@ struct DecTraits {
   static constexpr int kEPV = 16 / (int)sizeof(T);     // elements per 16-byte vector
   static constexpr int kLPR = kRowBytes / 16;          // lanes covering one row
   static constexpr int kRPI = 32 / kLPR;               // rows per warp-wide load
+  static constexpr int kNV = 8;                        // warp-wide loads per K (or V) part
+  static constexpr int kStageRows = 32;                // rows per copied stage
+  static constexpr int kWarpRows = kNV * kRPI;         // 16 (bf16 d=128), 32 (bf16 d=64), 8 (f32 d=128)
+  static constexpr int kSplit = kStageRows / kWarpRows;  // warps sharing a stage
   static constexpr int kStageBytes = kStageRows * kRowBytes;  // K or V part
-  static constexpr int kW = (2 * kStageBytes <= 8192) ? 8 : 6;        // consumer warps
-  static constexpr int kDepth = kStageBudget / (2 * kStageBytes * kW);  // buffers per warp
-  static constexpr int kStages = kW * kDepth;
+  static constexpr int kW = 12;                        // consumer warps
+  static constexpr int kGroups = kW / kSplit;          // warp groups, one stage each at a time
+  static constexpr int kDepth = kStageBudget / (2 * kStageBytes * kGroups);  // buffers per group
+  static constexpr int kStages = kGroups * kDepth;
   static constexpr int kConsumerThreads = kW * 32;
   static constexpr int kThreads = kConsumerThreads + 32;  // + one producer warp
-  static_assert(kLPR >= 8 && kLPR <= 32 && (kLPR & (kLPR - 1)) == 0, "unsupported row size");
+  static_assert(kLPR >= kNV && kLPR <= 32 && (kLPR & (kLPR - 1)) == 0, "unsupported row size");
+  static_assert(kStageRows % kWarpRows == 0 && kW % kSplit == 0, "stage split");
   static_assert(kDepth >= 1, "stage budget too small");
   static_assert(kConsumerThreads >= D, "one consumer thread per output dim");
   static constexpr size_t kBarOffset = (size_t)kStages * 2 * kStageBytes;
   static constexpr size_t kRedOffset = kBarOffset + 2 * kStages * 8;
-  static constexpr size_t kSmemBytes = kRedOffset + (2 * kW + kW * D) * 4 + 16;
+  // staged items: DecodeItem[kPreItems], int32 L_m[kPreItems], float q[kPreItems][D]
+  static constexpr size_t kMetaOffset = (kRedOffset + kBatch * (2 * kW + kW * D) * 4 + 16 + 15) / 16 * 16;
+  static constexpr size_t kLmOffset = kMetaOffset + sizeof(DecodeItem) * kPreItems;
+  static constexpr size_t kQOffset = kLmOffset + 4 * kPreItems;
+  static constexpr size_t kSmemBytes = kQOffset + 4 * (size_t)kPreItems * D;
   // partials that fit in the stage ring when it doubles as merge buffer
   static constexpr int kMergeCap = (int)(kBarOffset / ((D + 4) * 4));
 };
@@ -82,9 +104,12 @@ __device__ __forceinline__ int ld_cg(const int32_t* p) { return __ldcg(p); }
 // RSWA_TIMING builds record %globaltimer stamps per CTA (profiling aid).
 #ifdef RSWA_TIMING
 #define RSWA_STAMP(k) \
-  do { if (p.timing) p.timing[blockIdx.x * 8 + (k)] = global_ns(); } while (0)
+  do { if (p.timing) p.timing[blockIdx.x * 32 + (k)] = global_ns(); } while (0)
+#define RSWA_CYC(k) \
+  do { if (p.timing) p.timing[blockIdx.x * 32 + 16 + (k)] = clock64(); } while (0)
 #else
 #define RSWA_STAMP(k) do {} while (0)
+#define RSWA_CYC(k) do {} while (0)
 #endif
 
 __device__ __forceinline__ int atomic_add_acq_rel(int32_t* p, int v) {
@@ -103,14 +128,21 @@ __device__ __forceinline__ int atomic_add_release(int32_t* p, int v) {
 
 __device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 
+// Relaxed ticket: no ordering of its own (callers fence where needed).
+__device__ __forceinline__ int atomic_add_relaxed(int32_t* p, int v) {
+  int old;
+  asm volatile("atom.relaxed.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void griddep_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-// Valid cache rows of sequence b when the step counter reads T_now.
-__device__ __forceinline__ int valid_rows(const DecodeParams& p, int b, int T_now) {
-  const int Lm = p.Lm[b];
+// Valid cache rows of a sequence with Lm reference rows when the step
+// counter reads T_now.
+__device__ __forceinline__ int valid_rows(const DecodeParams& p, int Lm, int T_now) {
   const int len = p.full_mode ? Lm + T_now : Lm + min(p.n, T_now);
   return min(len, p.S_cap);
 }
@@ -120,6 +152,47 @@ __device__ __forceinline__ int valid_rows(const DecodeParams& p, int b, int T_no
 // shared memory (the stage ring, idle by then) with independent 16-byte
 // loads in one round, then thread `dim` folds them there.  Chunks of
 // `cap` partials bound the shared memory used.
+// The same for the slabs of up to two items at once (their partials together
+// fit in the buffer): one round of loads for both, then thread x*D + dim
+// folds item x.
+template <typename T, int D, int NT>
+__device__ __forceinline__ void merge_partials_joint(const DecodeParams& p, const DecodeItem& i0,
+                                                     const DecodeItem& i1, int n_its, int tid, float* buf) {
+  constexpr int RW = D + 4;
+  const int nv0 = i0.nparts * RW / 4;
+  const int nv = nv0 + (n_its > 1 ? i1.nparts * RW / 4 : 0);
+  const float4* s0 = reinterpret_cast<const float4*>(p.partials + (size_t)i0.part_first * RW);
+  const float4* s1 = reinterpret_cast<const float4*>(p.partials + (size_t)i1.part_first * RW);
+  float4* dst = reinterpret_cast<float4*>(buf);
+  for (int i = tid; i < nv; i += 4 * NT) {
+    float4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = i + u * NT;
+      if (j < nv) v[u] = __ldcg(j < nv0 ? s0 + j : s1 + (j - nv0));
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (i + u * NT < nv) dst[i + u * NT] = v[u];
+  }
+  named_barrier_sync(1, NT);
+  if (tid < n_its * D) {
+    const int x = tid / D, dd = tid % D;
+    const float* bx = buf + (x ? i0.nparts * RW : 0);
+    const int np = x ? i1.nparts : i0.nparts;
+    float M = -INFINITY;
+    for (int i = 0; i < np; ++i) M = fmaxf(M, bx[i * RW + D]);  // finite: the slab has rows
+    float acc = 0.f, L = 0.f;
+    for (int i = 0; i < np; ++i) {
+      const float w = exp2f(bx[i * RW + D] - M);  // exp2(-inf) = 0 for empty partials
+      acc = fmaf(w, bx[i * RW + dd], acc);
+      L = fmaf(w, bx[i * RW + D + 1], L);
+    }
+    store_elem(static_cast<T*>(p.o) + (size_t)(x ? i1.bh : i0.bh) * D + dd, acc / L);
+  }
+  named_barrier_sync(1, NT);
+}
+
 template <typename T, int D, int NT>
 __device__ __forceinline__ void merge_partials(const DecodeParams& p, const DecodeItem& item, int tid,
                                                float* buf, int cap) {
@@ -130,7 +203,17 @@ __device__ __forceinline__ void merge_partials(const DecodeParams& p, const Deco
     const int cn = min(cap, item.nparts - c0);
     const int nvec = cn * RW / 4;
     float4* dst = reinterpret_cast<float4*>(buf);
-    for (int i = tid; i < nvec; i += NT) dst[i] = __ldcg(src + (size_t)c0 * RW / 4 + i);
+    const float4* s0 = src + (size_t)c0 * RW / 4;
+    // independent loads, issued together: one L2 round trip per 4*NT vectors
+    for (int i = tid; i < nvec; i += 4 * NT) {
+      float4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (i + u * NT < nvec) v[u] = __ldcg(s0 + i + u * NT);
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (i + u * NT < nvec) dst[i + u * NT] = v[u];
+    }
     named_barrier_sync(1, NT);
     if (tid < D) {
       float Mc = M_run;
@@ -155,19 +238,23 @@ template <typename T, int D, bool APPEND>
 __global__ void __launch_bounds__(DecTraits<T, D>::kThreads, 1)
 decode_kernel(const __grid_constant__ DecodeParams p) {
   using Tr = DecTraits<T, D>;
-  constexpr int EPV = Tr::kEPV, LPR = Tr::kLPR, RPI = Tr::kRPI, NS = Tr::kStages;
+  constexpr int EPV = Tr::kEPV, LPR = Tr::kLPR, RPI = Tr::kRPI, NS = Tr::kStages, NV = Tr::kNV;
+  constexpr int kStageRows = Tr::kStageRows, WR = Tr::kWarpRows, GR = Tr::kGroups;
   constexpr int W = Tr::kW, NT = Tr::kConsumerThreads;
   constexpr int RB = Tr::kRowBytes, SB = Tr::kStageBytes;
 
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + Tr::kBarOffset);
   uint64_t* empty_bar = full_bar + NS;
-  float* red_m = reinterpret_cast<float*>(smem + Tr::kRedOffset);
-  float* red_l = red_m + W;
-  float* red_o = red_l + W;
-  volatile int* s_flag = reinterpret_cast<volatile int*>(red_o + W * D);  // [2]
+  float* red_m = reinterpret_cast<float*>(smem + Tr::kRedOffset);  // [kBatch][W]
+  float* red_l = red_m + kBatch * W;                                // [kBatch][W]
+  float* red_o = red_l + kBatch * W;                                // [kBatch][W][D]
+  volatile int* s_flag = reinterpret_cast<volatile int*>(red_o + kBatch * W * D);  // [2]
   volatile int* s_abort = s_flag + 2;
   volatile int* s_T = s_flag + 3;
+  DecodeItem* s_items = reinterpret_cast<DecodeItem*>(smem + Tr::kMetaOffset);
+  int* s_lm = reinterpret_cast<int*>(smem + Tr::kLmOffset);
+  float* s_q = reinterpret_cast<float*>(smem + Tr::kQOffset);
   float* merge_buf = reinterpret_cast<float*>(smem);  // the stage ring, once drained
 
   const int warp = threadIdx.x >> 5;
@@ -177,26 +264,80 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
     RSWA_STAMP(0);
     for (int s = 0; s < NS; ++s) {
       mbar_init(smem_u32(&full_bar[s]), 1);
-      mbar_init(smem_u32(&empty_bar[s]), 32);  // every lane of the owning warp
+      mbar_init(smem_u32(&empty_bar[s]), 32 * Tr::kSplit);  // every lane of the owning group
     }
     *s_abort = 0;
     fence_barrier_init();
   }
-  // The plan is written by the host before any launch that uses it, so it
-  // can be read before waiting on the previous kernel.  So can an L2
-  // prefetch of the rows this CTA will stream: L2 is coherent, so a row the
-  // previous kernel still writes is simply fetched again later.  Bounded so
-  // that all CTAs together stay well inside L2.
+  // The plan and the reference lengths are written by host copies ordered
+  // before any launch that uses them, so they can be read (and the first
+  // kPreItems items staged in shared memory) before waiting on the previous
+  // kernel.  So can an L2 prefetch of the rows this CTA will stream: L2 is
+  // coherent, so a row the previous kernel still writes is simply fetched
+  // again later.
   const int it_begin = p.cta_begin[blockIdx.x];
   const int it_end = p.cta_begin[blockIdx.x + 1];
+  const int n_pre = min(it_end - it_begin, kPreItems);
+  if ((int)threadIdx.x < n_pre) {
+    const DecodeItem item = p.items[it_begin + threadIdx.x];
+    s_items[threadIdx.x] = item;
+    s_lm[threadIdx.x] = p.Lm[item.bh / p.H];
+  }
   __syncthreads();
   griddep_launch_dependents();
+  auto item_at = [&](int it) -> DecodeItem {
+    const int li = it - it_begin;
+    return li < kPreItems ? s_items[li] : p.items[it];
+  };
+  auto lm_at = [&](int it, const DecodeItem& item) -> int {
+    const int li = it - it_begin;
+    return li < kPreItems ? s_lm[li] : p.Lm[item.bh / p.H];
+  };
+  // Stage issue, in stage order g over the span: (it, j) is the next stage.
+  int p_it = it_begin, p_j = 0;
+  uint32_t g = 0;
+  auto issue = [&](const DecodeItem& item, int j) {
+    const int slot = g % NS;
+    const int nr = min(kStageRows, item.rows - j * kStageRows);
+    const uint32_t bytes = (uint32_t)(nr * RB);
+    const size_t row = (size_t)item.bh * p.S_cap + item.row0 + (size_t)j * kStageRows;
+    const uint32_t fb = smem_u32(&full_bar[slot]);
+    uint8_t* dst = smem + (size_t)slot * 2 * SB;
+    mbar_arrive_expect_tx(fb, 2 * bytes);
+    bulk_g2s(smem_u32(dst), static_cast<const uint8_t*>(p.kc) + row * RB, bytes, fb);
+    bulk_g2s(smem_u32(dst + SB), static_cast<const uint8_t*>(p.vc) + row * RB, bytes, fb);
+    if (g == 0) RSWA_STAMP(2);
+    ++g;
+  };
+  // Reference rows are written only by the reference load, whose kernel
+  // fences its writes before it retires, so with ref_stable the leading
+  // stages made only of reference rows are copied before the dependency
+  // wait, into buffers that are still free (g < NS).  Output rows (the
+  // ring) may be written by the previous kernel and are copied after it.
+  if (warp == W && lane == 0 && p.ref_stable) {
+    while (p_it < it_end && g < (uint32_t)NS) {
+      const DecodeItem item = item_at(p_it);
+      const int nst = (item.rows + kStageRows - 1) / kStageRows;
+      if (p_j >= nst) {
+        ++p_it;
+        p_j = 0;
+        continue;
+      }
+      const int nr = min(kStageRows, item.rows - p_j * kStageRows);
+      if (item.row0 + p_j * kStageRows + nr > lm_at(p_it, item)) break;
+      issue(item, p_j);
+      ++p_j;
+    }
+  }
+  // L2 prefetch of the rows not copied early (bounded so that all CTAs
+  // together stay well inside L2).
   if (warp == W && lane == 0) {
     long long budget = kPrefetchBytes;
-    for (int it = it_begin; it < it_end && budget > 0; ++it) {
-      const DecodeItem item = p.items[it];
-      const size_t off = ((size_t)item.bh * p.S_cap + item.row0) * RB;
-      const long long bytes = min((long long)item.rows * RB, budget);
+    for (int it = p_it; it < it_end && budget > 0; ++it) {
+      const DecodeItem item = item_at(it);
+      const int r0 = it == p_it ? min(p_j * kStageRows, item.rows) : 0;
+      const size_t off = ((size_t)item.bh * p.S_cap + item.row0 + r0) * RB;
+      const long long bytes = min((long long)(item.rows - r0) * RB, budget);
       for (long long o = 0; o < bytes; o += kPrefetchChunk) {
         const uint32_t nb = (uint32_t)min((long long)kPrefetchChunk, bytes - o);
         bulk_prefetch_l2(static_cast<const uint8_t*>(p.kc) + off + o, nb);
@@ -205,36 +346,36 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
       budget -= bytes;
     }
   }
+#ifdef RSWA_TIMING
+  if (warp == W - 1 && lane == 0 && it_begin < it_end) {  // when the first stage lands
+    mbar_wait_bounded(smem_u32(&full_bar[0]), 0);
+    RSWA_STAMP(12);
+  }
+#endif
   griddep_wait();  // everything below may read what the previous kernel wrote
   if (threadIdx.x == 0) RSWA_STAMP(1);
 
   // ------------------------------------------------------------ producer
   if (warp == W) {
     if (lane != 0) return;
-    uint32_t g = 0;
     bool ok = true;
-    for (int it = it_begin; it < it_end && ok; ++it) {
-      const DecodeItem item = p.items[it];
+    while (p_it < it_end && ok) {
+      const DecodeItem item = item_at(p_it);
       const int nst = (item.rows + kStageRows - 1) / kStageRows;
-      const uint8_t* kb = static_cast<const uint8_t*>(p.kc) + ((size_t)item.bh * p.S_cap + item.row0) * RB;
-      const uint8_t* vb = static_cast<const uint8_t*>(p.vc) + ((size_t)item.bh * p.S_cap + item.row0) * RB;
-      for (int j = 0; j < nst; ++j, ++g) {
-        const int slot = g % NS;
-        if (*s_abort || !mbar_wait_bounded(smem_u32(&empty_bar[slot]), ((g / NS) & 1) ^ 1)) {
-          flag_error(p.err, kErrWaitTimeout);
-          *s_abort = 1;
-          ok = false;
-          break;
-        }
-        const int nr = min(kStageRows, item.rows - j * kStageRows);
-        const uint32_t bytes = (uint32_t)(nr * RB);
-        const uint32_t fb = smem_u32(&full_bar[slot]);
-        uint8_t* dst = smem + (size_t)slot * 2 * SB;
-        mbar_arrive_expect_tx(fb, 2 * bytes);
-        bulk_g2s(smem_u32(dst), kb + (size_t)j * kStageRows * RB, bytes, fb);
-        bulk_g2s(smem_u32(dst + SB), vb + (size_t)j * kStageRows * RB, bytes, fb);
-        if (g == 0) RSWA_STAMP(2);
+      if (p_j >= nst) {
+        ++p_it;
+        p_j = 0;
+        continue;
       }
+      const int slot = g % NS;
+      if (*s_abort || !mbar_wait_bounded(smem_u32(&empty_bar[slot]), ((g / NS) & 1) ^ 1)) {
+        flag_error(p.err, kErrWaitTimeout);
+        *s_abort = 1;
+        ok = false;
+        break;
+      }
+      issue(item, p_j);
+      ++p_j;
     }
     // Drain: never leave the CTA with bulk copies still writing shared memory.
     const uint32_t first = g > (uint32_t)NS ? g - NS : 0;
@@ -246,15 +387,36 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
   }
 
   // ------------------------------------------------------------ consumers
+  // The step counter and the queries of the staged items are outputs of
+  // earlier kernels: one round of independent loads.
   if (threadIdx.x == 0) *s_T = ld_cg(p.T);
+  {
+    constexpr int VPR = D / EPV;  // 16-byte vectors per query row
+    for (int x = threadIdx.x; x < n_pre * VPR; x += NT) {
+      const int i = x / VPR, v = x % VPR;
+      const uint4 qu =
+          *reinterpret_cast<const uint4*>(static_cast<const T*>(p.q) + (size_t)s_items[i].bh * D + v * EPV);
+      float f[EPV];
+      Vec16<T>::unpack(qu, f);
+#pragma unroll
+      for (int e = 0; e < EPV; ++e) s_q[i * D + v * EPV + e] = f[e] * p.scale_log2;
+    }
+  }
   named_barrier_sync(1, NT);
+  if (threadIdx.x == 0) {
+    RSWA_STAMP(8);
+    RSWA_CYC(0);
+  }
   const int T0 = *s_T;
   const int T_step = T0 + (APPEND ? 1 : 0);  // outputs in the cache for this step
   // Launch ticket, taken right after the read of T but only looked at at the
   // end: the CTA holding the last ticket knows every CTA has read T, so it
   // may advance T (the others keep their copy).
+  // (Relaxed: this thread's read of T has already returned and been used.)
   int launch_ticket = 0;
-  if (APPEND && threadIdx.x == 0) launch_ticket = atomic_add_release(p.done, 1);
+  if (APPEND && threadIdx.x == 0) launch_ticket = atomic_add_relaxed(p.done, 1);
+  const int group = warp / Tr::kSplit;            // stage group of this warp
+  const int part_row = (warp % Tr::kSplit) * WR;  // its first row inside a stage
   const int grp = lane / LPR;   // which of the RPI rows of a warp-wide load
   const int sub = lane % LPR;   // which 16-byte slice of the row
   const int tid = threadIdx.x;  // 0 .. NT-1
@@ -262,42 +424,55 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
   int pend0 = -1, pend1 = -1;   // split items (at most the first and last of the span)
   int tk0 = 0, tk1 = 0;         // their tickets (valid in thread 0)
 
-  for (int it = it_begin; it < it_end; ++it) {
-    const DecodeItem item = p.items[it];
+  for (int it0 = it_begin; it0 < it_end; it0 += kBatch) {
+   const int nb = min(kBatch, it_end - it0);
+   for (int x = 0; x < nb; ++x) {
+    const int it = it0 + x;
+    const int li = it - it_begin;
+    const DecodeItem item = li < kPreItems ? s_items[li] : p.items[it];
     const int b = item.bh / p.H;
+    const int Lm_b = li < kPreItems ? s_lm[li] : p.Lm[b];
     const int T_now = T_step;
-    const int len = valid_rows(p, b, T_now);
+    const int len = valid_rows(p, Lm_b, T_now);
     const int live = max(0, min(len - item.row0, item.rows));  // rows to attend
     const int nst = (item.rows + kStageRows - 1) / kStageRows;  // stages streamed
     if (tid == 0 && item.last && len > item.row0 + item.rows) flag_error(p.err, kErrPlanShort);
 
     int slot_row = -1;
     if (APPEND) {
-      const int Lm = p.Lm[b];
       if (p.full_mode) {
-        if (T_now <= p.T_cap) slot_row = Lm + T_now - 1;
+        if (T_now <= p.T_cap) slot_row = Lm_b + T_now - 1;
         else if (tid == 0 && item.row0 == 0) flag_error(p.err, kErrCapacity);
       } else {
-        slot_row = Lm + (T_now - 1) % p.n;
+        slot_row = Lm_b + (T_now - 1) % p.n;
       }
     }
 
     float qf[EPV], of[EPV];
-    {
+    if (li < kPreItems) {
+#pragma unroll
+      for (int e = 0; e < EPV; e += 4) {
+        const float4 q4 = *reinterpret_cast<const float4*>(s_q + li * D + sub * EPV + e);
+        qf[e] = q4.x;
+        qf[e + 1] = q4.y;
+        qf[e + 2] = q4.z;
+        qf[e + 3] = q4.w;
+      }
+    } else {
       const uint4 qu =
           *reinterpret_cast<const uint4*>(static_cast<const T*>(p.q) + (size_t)item.bh * D + sub * EPV);
       Vec16<T>::unpack(qu, qf);
 #pragma unroll
-      for (int e = 0; e < EPV; ++e) {
-        qf[e] *= p.scale_log2;
-        of[e] = 0.f;
-      }
+      for (int e = 0; e < EPV; ++e) qf[e] *= p.scale_log2;
     }
+#pragma unroll
+    for (int e = 0; e < EPV; ++e) of[e] = 0.f;
     float m = -INFINITY, l = 0.f;
 
-    // this warp's stages of the item: global stage index = warp (mod W)
-    const int j0 = (warp - (int)(gctr % W) + W) % W;
-    for (int j = j0; j < nst; j += W) {
+    // this warp group's stages of the item: global stage index = group (mod GR)
+    const int j0 = (group - (int)(gctr % GR) + GR) % GR;
+    if (tid == 0 && it == it_begin) RSWA_CYC(1);
+    for (int j = j0; j < nst; j += GR) {
       const uint32_t gs = gctr + j;
       const int slot = gs % NS;
       if (*s_abort || !mbar_wait_bounded(smem_u32(&full_bar[slot]), (gs / NS) & 1)) {
@@ -307,17 +482,21 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
         }
         break;
       }
-      if (gs == 0 && lane == 0) RSWA_STAMP(3);
-      const int nr = min(kStageRows, live - j * kStageRows);  // may be <= 0: nothing to attend
+      if (gs == 0 && lane == 0) {
+        RSWA_STAMP(3);
+        RSWA_CYC(2);
+      }
+      // this warp's rows of the stage: [part_row, part_row + WR)
+      const int nr = min(WR, live - j * kStageRows - part_row);  // may be <= 0: nothing to attend
       if (nr > 0) {
-        const int r_base = item.row0 + j * kStageRows;
-        const uint8_t* Ks = smem + (size_t)slot * 2 * SB;
+        const int r_base = item.row0 + j * kStageRows + part_row;
+        const uint8_t* Ks = smem + (size_t)slot * 2 * SB + part_row * RB;
         const uint8_t* Vs = Ks + SB;
-        float part[LPR];
+        float part[NV];
         int sub_k = -1;
         uint4 vsub = make_uint4(0, 0, 0, 0);
 #pragma unroll
-        for (int k = 0; k < LPR; ++k) {
+        for (int k = 0; k < NV; ++k) {
           const int row = k * RPI + grp;
           uint4 u = *reinterpret_cast<const uint4*>(Ks + row * RB + sub * 16);
           if (APPEND && r_base + row == slot_row) {
@@ -337,10 +516,13 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
           for (int e = 0; e < EPV; ++e) acc = fmaf(qf[e], f[e], acc);
           part[k] = acc;
         }
-        // Transposed butterfly: after log2(LPR) steps lane `sub` of each row
-        // group holds the full dot product of row sub*RPI + grp.
+        if (gs == 0 && lane == 0) RSWA_CYC(3);
+        // Transposed butterfly over the low log2(NV) lane bits: lane `sub`
+        // keeps value sub % NV summed over its NV-lane group; then plain
+        // shuffles sum the groups of the row, so every lane holds the full
+        // dot product of row (sub % NV) * RPI + grp.
 #pragma unroll
-        for (int mk = LPR / 2; mk >= 1; mk >>= 1) {
+        for (int mk = NV / 2; mk >= 1; mk >>= 1) {
           const bool upper = (sub & mk) != 0;
 #pragma unroll
           for (int i = 0; i < mk; ++i) {
@@ -349,8 +531,12 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
             part[i] = keep + __shfl_xor_sync(0xffffffffu, send, mk);
           }
         }
-        const int my_row = sub * RPI + grp;
+#pragma unroll
+        for (int mk = NV; mk < LPR; mk <<= 1) part[0] += __shfl_xor_sync(0xffffffffu, part[0], mk);
+        const int my_row = (sub % NV) * RPI + grp;
         const bool valid = my_row < nr;
+        const bool owner = sub < NV;  // one lane per row adds to the sum
+        if (gs == 0 && lane == 0) RSWA_CYC(4);
         const float sc = valid ? part[0] : -INFINITY;
         float mx = sc;
 #pragma unroll
@@ -358,11 +544,12 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
         const float m_new = fmaxf(m, mx);  // finite: the stage has a valid row
         const float corr = exp2f(m - m_new);
         const float pr = valid ? exp2f(sc - m_new) : 0.f;
-        l = l * corr + pr;
+        l = l * corr + (owner ? pr : 0.f);
+        if (gs == 0 && lane == 0) RSWA_CYC(5);
 #pragma unroll
         for (int e = 0; e < EPV; ++e) of[e] *= corr;
 #pragma unroll
-        for (int k = 0; k < LPR; ++k) {
+        for (int k = 0; k < NV; ++k) {
           const int row = k * RPI + grp;
           const float pk = __shfl_sync(0xffffffffu, pr, grp * LPR + k);
           if (row < nr) {
@@ -376,12 +563,16 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
         }
         m = m_new;
       }
+      if (gs == 0 && lane == 0) {
+        RSWA_STAMP(9);
+        RSWA_CYC(6);
+      }
       // Each lane releases the buffer after its own shared-memory reads.
       mbar_arrive(smem_u32(&empty_bar[slot]));
     }
     gctr += nst;
 
-    // ---- merge the consumer warps of this item
+    // ---- this warp's partial of item x: (m, l, o) into shared memory
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
 #pragma unroll
@@ -391,48 +582,63 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
     }
     if (grp == 0) {
 #pragma unroll
-      for (int e = 0; e < EPV; ++e) red_o[warp * D + sub * EPV + e] = of[e];
+      for (int e = 0; e < EPV; ++e) red_o[(x * W + warp) * D + sub * EPV + e] = of[e];
     }
     if (lane == 0) {
-      red_m[warp] = m;
-      red_l[warp] = l;
+      red_m[x * W + warp] = m;
+      red_l[x * W + warp] = l;
     }
+   }
+    // ---- merge the consumer warps of the batch's items (thread x*D + d)
     named_barrier_sync(1, NT);
-    if (tid < D) {
+    if (tid < nb * D) {
+      const int x = tid / D, dd = tid % D;
+      const DecodeItem item = item_at(it0 + x);
       float M = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < W; ++w) M = fmaxf(M, red_m[w]);
+      for (int w = 0; w < W; ++w) M = fmaxf(M, red_m[x * W + w]);
       float acc = 0.f, Ls = 0.f;
 #pragma unroll
       for (int w = 0; w < W; ++w) {
-        const float mw = red_m[w];
+        const float mw = red_m[x * W + w];
         const float wt = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
-        acc = fmaf(wt, red_o[w * D + tid], acc);
-        Ls = fmaf(wt, red_l[w], Ls);
+        acc = fmaf(wt, red_o[(x * W + w) * D + dd], acc);
+        Ls = fmaf(wt, red_l[x * W + w], Ls);
       }
       if (item.nparts == 1) {
-        store_elem(static_cast<T*>(p.o) + (size_t)item.bh * D + tid, acc / Ls);
+        store_elem(static_cast<T*>(p.o) + (size_t)item.bh * D + dd, acc / Ls);
       } else {
         float* P = p.partials + (size_t)item.part * (D + 4);
-        P[tid] = acc;
-        if (tid == 0) {
+        P[dd] = acc;
+        if (dd == 0) {
           P[D] = M;
           P[D + 1] = Ls;
         }
       }
     }
-    named_barrier_sync(1, NT);  // partial written; red_* are reused by the next item
-    if (item.nparts > 1) {
-      // Ticket with release semantics right away (after the barrier, so it
-      // covers every thread's partial writes); its value is read at the end.
-      if (pend0 < 0) {
-        pend0 = it;
-        if (tid == 0) tk0 = atomic_add_release(p.tickets + item.bh, 1);
-      } else if (pend1 < 0) {
-        pend1 = it;
-        if (tid == 0) tk1 = atomic_add_release(p.tickets + item.bh, 1);
-      } else if (tid == 0) {  // a span has at most two split items
-        flag_error(p.err, kErrPlanShort);
+    named_barrier_sync(1, NT);  // partials written; red_* are reused by the next batch
+    if (tid == 0 && it0 == it_begin) RSWA_STAMP(10);
+    // Tickets of the batch's split items right away: one release fence
+    // (after the barrier, so it covers every thread's partial writes), then
+    // relaxed increments in flight together; their values are read at the end.
+    bool fenced = false;
+    for (int x = 0; x < nb; ++x) {
+      const int it = it0 + x;
+      const DecodeItem item = item_at(it);
+      if (item.nparts > 1) {
+        if (tid == 0 && !fenced) {
+          fence_acq_rel_gpu();
+          fenced = true;
+        }
+        if (pend0 < 0) {
+          pend0 = it;
+          if (tid == 0) tk0 = atomic_add_relaxed(p.tickets + item.bh, 1);
+        } else if (pend1 < 0) {
+          pend1 = it;
+          if (tid == 0) tk1 = atomic_add_relaxed(p.tickets + item.bh, 1);
+        } else if (tid == 0) {  // a span has at most two split items
+          flag_error(p.err, kErrPlanShort);
+        }
       }
     }
   }
@@ -441,19 +647,33 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
   // ---- split items: the CTA holding the last ticket of a slab merges it.
   if (tid == 0) {
     int l0 = 0, l1 = 0;
-    if (pend0 >= 0) l0 = tk0 == p.items[pend0].nparts - 1;
-    if (pend1 >= 0) l1 = tk1 == p.items[pend1].nparts - 1;
+    if (pend0 >= 0) l0 = tk0 == item_at(pend0).nparts - 1;
+    if (pend1 >= 0) l1 = tk1 == item_at(pend1).nparts - 1;
     if (l0 || l1) fence_acq_rel_gpu();  // acquire the other CTAs' partials
     s_flag[0] = l0;
     s_flag[1] = l1;
+    RSWA_STAMP(11);
   }
   named_barrier_sync(1, NT);
-  for (int i = 0; i < 2; ++i) {
-    if (!s_flag[i]) continue;  // uniform across the CTA
-    const DecodeItem item = p.items[i == 0 ? pend0 : pend1];
-    merge_partials<T, D, NT>(p, item, tid, merge_buf, Tr::kMergeCap);
-    if (tid == 0) p.tickets[item.bh] = 0;
-    named_barrier_sync(1, NT);
+  {
+    // the slabs this CTA merges (uniform across the CTA): m0, then m1
+    const int f0 = s_flag[0], f1 = s_flag[1];
+    const int nm = f0 + f1;
+    if (nm > 0) {
+      const DecodeItem m0 = item_at(f0 ? pend0 : pend1);
+      const DecodeItem m1 = item_at(pend1 >= 0 ? pend1 : pend0);
+      if (m0.nparts + (nm > 1 ? m1.nparts : 0) <= Tr::kMergeCap) {
+        merge_partials_joint<T, D, NT>(p, m0, m1, nm, tid, merge_buf);
+      } else {
+        merge_partials<T, D, NT>(p, m0, tid, merge_buf, Tr::kMergeCap);
+        if (nm > 1) merge_partials<T, D, NT>(p, m1, tid, merge_buf, Tr::kMergeCap);
+      }
+      if (tid == 0) {
+        RSWA_STAMP(13);
+        p.tickets[m0.bh] = 0;
+        if (nm > 1) p.tickets[m1.bh] = 0;
+      }
+    }
   }
 
   if (tid == 0) RSWA_STAMP(5);

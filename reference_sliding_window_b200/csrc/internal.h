@@ -74,6 +74,7 @@ struct DecodeParams {
   int32_t* tickets;
   int32_t* done;
   int32_t* err;
+  int ref_stable;        // 1: the reference rows are final (see decode.cu); 0: read after the wait
   float scale_log2;      // softmax scale * log2(e)
   unsigned long long* timing;  // profiling stamps (RSWA_TIMING builds), may be null
 };
