@@ -570,6 +570,7 @@ extern "C" rswa_status rswa_masked_forward(const void* Q, const void* K, const v
   p.D = d;
   const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)d);
   p.scale_log2 = sc * 1.4426950408889634f;
+  p.timing = g_timing;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (dtype == RSWA_BF16 && d == 128) {
     RSWA_CUDA(launch_masked_forward_tc(p, s), "masked forward tensor-core kernel");

@@ -114,6 +114,7 @@ struct MaskedParams {
   void* O;
   int L, L_m, n, H, D;
   float scale_log2;
+  unsigned long long* timing;  // profiling stamps (RSWA_TIMING builds), may be null
 };
 // Sets the thread-local message returned by rswa_last_error().
 void set_last_error(const char* prefix, const char* msg);

@@ -13,18 +13,30 @@
 // * The key tiles a query tile needs are the reference tiles [0, ceil(L_m/128))
 //   plus the 2-3 tiles of its causal band; every other tile is fully masked
 //   and skipped.  Only tiles that are not fully visible are masked per element.
-// * Warp 0 lane 0 loads Q once and streams K/V tiles with TMA (128B-swizzled
-//   boxes of 128 rows x 64 columns) into a 2-stage ring.  Warp 1 owns the
-//   tensor memory (512 columns: S double-buffered, O) and one lane issues the
-//   MMAs: S_j = Q K_j^T into TMEM, then O += P_{j-1} V_{j-1}, so the QK^T of
-//   tile j overlaps the softmax of tile j-1.
-// * Warps 2.. run the softmax, kSplit threads per query row: warps w, w+4, ...
-//   read the same TMEM lanes, each taking 128/kSplit columns.  The parts of a
-//   row exchange their maxima through shared memory (one named barrier per
-//   tile), form p = 2^(s*scale*log2e - m), write their part of P (bf16,
-//   128B-swizzled) for the PV MMA, and rescale their part of O in TMEM
-//   only when the row maximum grew by more than 2^8 since the last rescale
-//   (the stale maximum keeps every exponent <= 2^8, exact in float32).
+// * Warp 0 lane 0 loads Q once and streams K tiles with TMA (128B-swizzled
+//   boxes of 128 rows x 64 columns) into a 3-stage ring whose stages free as
+//   soon as their QK^T MMA completes; warp 10 lane 0 streams V tiles into a
+//   2-stage ring freed by the PV MMAs.  Separate rings and producers keep a
+//   K load from waiting behind a V stage, so copies run two tiles ahead of
+//   the MMAs and their latency stays hidden.  Warp 1 owns the
+//   tensor memory (512 columns: S, O_A, O_B, P double-buffered) and one lane
+//   issues the MMAs: S_j = Q K_j^T into TMEM, then the PV products of tile
+//   j-1 with P read from TMEM, so the QK^T of tile j overlaps the softmax of
+//   tile j-1.  Keeping P in tensor memory leaves shared memory to the Q, K
+//   and V operands: at N = 128 an MMA with both operands in shared memory
+//   already takes all of its bandwidth.
+// * Warps 2..9 run the softmax, two threads per query row: warps w and w+4
+//   read the same TMEM lanes, one the keys 0..63 of each tile, the other the
+//   keys 64..127.  Each half keeps its own running maximum and sum and its
+//   own output accumulator (O_A += P[:, 0:64] V[0:64], O_B += P[:, 64:128]
+//   V[64:128]), so the halves never wait for each other inside the loop;
+//   the two are combined by the log-sum-exp rule once, at the end.  A thread
+//   forms p = 2^(s*scale*log2e - m), stores its half of P (bf16 pairs) into
+//   the tile's P buffer in TMEM, and rescales its O row only when its
+//   maximum grew by more than 2^8 since the last rescale (the stale maximum
+//   keeps every exponent <= 2^8, exact in float32).  So the softmax of tile
+//   j waits for the PV MMAs of tile j-1 only when it rescales; otherwise
+//   only for those of tile j-2 (the P buffer it reuses).
 // * Every wait is bounded; on a timeout the kernel marks its rows with NaN,
 //   drains its copies and MMAs, frees its tensor memory and returns.
 
@@ -49,27 +61,25 @@ namespace tc {
 
 constexpr int kTile = 128;     // query and key tile
 constexpr int kD = 128;        // head dim
-#ifndef RSWA_TC_SPLIT
-#define RSWA_TC_SPLIT 2
-#endif
-constexpr int kSplit = RSWA_TC_SPLIT;  // softmax threads per query row
+constexpr int kSplit = 2;              // softmax threads per query row
 constexpr int kHalf = 128 / kSplit;    // columns per softmax thread
 constexpr int kBox = 64;       // columns per 128B-swizzled box (bf16)
 constexpr int kBoxBytes = kTile * kBox * 2;      // 16 KB
 constexpr int kTileBytes = 2 * kBoxBytes;        // 32 KB: 128 rows x 128 cols
-constexpr int kKV = 2;                           // K/V ring stages
+constexpr int kKS = 3;                           // K ring stages
+constexpr int kVS = 2;                           // V ring stages
 constexpr int kSoftmaxThreads = 128 * kSplit;    // warps 2 .. 2 + 4*kSplit - 1
-constexpr int kThreads = 64 + kSoftmaxThreads;   // producer, MMA, softmax
+constexpr int kVWarp = 2 + kSoftmaxThreads / 32;  // V producer warp (after the softmax warps)
+constexpr int kThreads = 64 + kSoftmaxThreads + 32;  // K producer, MMA, softmax, V producer
 constexpr int kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
+constexpr uint32_t kColS = 0, kColOA = 128, kColOB = 256, kColP0 = 384, kColP1 = 448;  // P: bf16 pairs
 
 // Shared memory map (offsets from a 1024-byte aligned base).
 constexpr int kSmQ = 0;
 constexpr int kSmK = kSmQ + kTileBytes;
-constexpr int kSmV = kSmK + kKV * kTileBytes;
-constexpr int kSmP = kSmV + kKV * kTileBytes;
-constexpr int kSmRed = kSmP + kTileBytes;        // float rmax[2][kSplit][128], lsum[kSplit][128]
-constexpr int kSmBar = kSmRed + (2 * kSplit * kTile + kSplit * kTile) * 4;
+constexpr int kSmV = kSmK + kKS * kTileBytes;
+constexpr int kSmRed = kSmV + kVS * kTileBytes;  // float mfin[kSplit][128], lfin[kSplit][128]
+constexpr int kSmBar = kSmRed + 2 * kSplit * kTile * 4;
 constexpr int kSmBytes = kSmBar + 256 + 1024;    // + slack for 1024-byte alignment
 
 // Instruction descriptor of tcgen05.mma kind::f16: bf16 A and B, float32 D,
@@ -99,6 +109,16 @@ __device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}"
       ::"r"(tmem_d), "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(0), "r"(0), "r"(0), "r"(0)
+      : "memory");
+}
+
+// The same with A (M x K, bf16 pairs along the columns) read from TMEM.
+__device__ __forceinline__ void mma_bf16_ta(uint32_t tmem_d, uint32_t tmem_a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}"
+      ::"r"(tmem_d), "r"(tmem_a), "l"(b), "r"(idesc), "r"(acc), "r"(0), "r"(0), "r"(0), "r"(0)
       : "memory");
 }
 
@@ -171,6 +191,17 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
       : "memory");
 }
 
+// kHalf/2 consecutive TMEM columns of this thread's lane from packed words.
+__device__ __forceinline__ void tmem_st_pairs(uint32_t taddr, const uint32_t* w) {
+#pragma unroll
+  for (int c = 0; c < kHalf / 2; c += 16) {
+    float v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(w[c + i]);
+    tmem_st16(taddr + c, v);
+  }
+}
+
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -207,7 +238,17 @@ struct TcParams {
   __nv_bfloat16* O;
   int L, L_m, n, H, n_qtiles;
   float scale_log2;
+  unsigned long long* timing;  // RSWA_TIMING builds: per-tile cycle stamps of CTA 0
 };
+
+// RSWA_TIMING builds record clock64 stamps of CTA 0 for its first 32 tiles:
+// slot [j][k], k < 8 by softmax warp 2 lane 0, k >= 8 by the MMA thread.
+#ifdef RSWA_TIMING
+#define TC_CYC(j, k) \
+  do { if (p.timing && blockIdx.x == 0 && (j) < 32) p.timing[(j) * 16 + (k)] = clock64(); } while (0)
+#else
+#define TC_CYC(j, k) do {} while (0)
+#endif
 
 // Key tiles of query tile at q0: [0, A) then [B0, B1] (B0 > A-1 or empty).
 struct TileRange {
@@ -235,8 +276,8 @@ __device__ __forceinline__ int tile_at(const TileRange& r, int j) { return j < r
 
 // Barrier slots (8 bytes each).
 enum : int {
-  kBarQ = 0, kBarKFull = 1, kBarVFull = 3, kBarKVFree = 5, kBarSFull = 7, kBarSFree = 9,
-  kBarPFull = 11, kBarODone = 12, kBarFinal = 13, kSlotTmem = 14, kSlotAbort = 15
+  kBarQ = 0, kBarKFull = 1, kBarKFree = 4, kBarVFull = 7, kBarVFree = 9, kBarSFull = 11, kBarSFree = 12,
+  kBarPFull = 13, kBarPFree = 15, kBarFinal = 17, kSlotTmem = 18, kSlotAbort = 19
 };
 
 // One thread's half row of an S tile (64 columns starting at col0):
@@ -287,8 +328,8 @@ __global__ void __launch_bounds__(kThreads, 1) masked_tc_kernel(const __grid_con
   auto B = [&](int slot) { return bar0 + 8u * slot; };
   volatile uint32_t* s_tmem = reinterpret_cast<volatile uint32_t*>(&bars[kSlotTmem]);
   volatile int* s_abort = reinterpret_cast<volatile int*>(&bars[kSlotAbort]);
-  float* rmax = reinterpret_cast<float*>(smem + kSmRed);  // [parity][part][row]
-  float* lsum = rmax + 2 * kSplit * kTile;                 // [part][row]
+  float* mfin = reinterpret_cast<float*>(smem + kSmRed);  // [half][row]: final maxima
+  float* lfin = mfin + kSplit * kTile;                     // [half][row]: final sums
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -304,17 +345,20 @@ __global__ void __launch_bounds__(kThreads, 1) masked_tc_kernel(const __grid_con
 
   if (threadIdx.x == 0) {
     mbar_init(B(kBarQ), 1);
-    for (int s = 0; s < kKV; ++s) {
+    for (int s = 0; s < kKS; ++s) {
       mbar_init(B(kBarKFull + s), 1);
+      mbar_init(B(kBarKFree + s), 1);
+    }
+    for (int s = 0; s < kVS; ++s) {
       mbar_init(B(kBarVFull + s), 1);
-      mbar_init(B(kBarKVFree + s), 1);
+      mbar_init(B(kBarVFree + s), 1);
     }
+    mbar_init(B(kBarSFull), 1);
+    mbar_init(B(kBarSFree), kSoftmaxThreads);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(B(kBarSFull + s), 1);
-      mbar_init(B(kBarSFree + s), kSoftmaxThreads);
+      mbar_init(B(kBarPFull + s), kSoftmaxThreads);
+      mbar_init(B(kBarPFree + s), 1);
     }
-    mbar_init(B(kBarPFull), kSoftmaxThreads);
-    mbar_init(B(kBarODone), 1);
     mbar_init(B(kBarFinal), 1);
     *s_abort = 0;
     fence_barrier_init();
@@ -330,71 +374,76 @@ __global__ void __launch_bounds__(kThreads, 1) masked_tc_kernel(const __grid_con
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
 
-  if (warp == 0) {
-    // ---------------------------------------------------------- producer
+  if (warp == 0 || warp == kVWarp) {
+    // ---------------------------------------------------------- producers
+    // warp 0: Q, then the K ring; warp kVWarp: the V ring
     if (lane == 0) {
-      mbar_arrive_expect_tx(B(kBarQ), kTileBytes);
-      tma_load_3d(sbase + kSmQ, &p.tmQ, 0, h, q0, B(kBarQ));
-      tma_load_3d(sbase + kSmQ + kBoxBytes, &p.tmQ, kBox, h, q0, B(kBarQ));
+      const bool is_k = warp == 0;
+      const int ns = is_k ? kKS : kVS;
+      const uint32_t full0 = B(is_k ? kBarKFull : kBarVFull), free0 = B(is_k ? kBarKFree : kBarVFree);
+      const uint32_t dst0 = sbase + (is_k ? kSmK : kSmV);
+      const CUtensorMap* map = is_k ? &p.tmK : &p.tmV;
+      if (is_k) {
+        mbar_arrive_expect_tx(B(kBarQ), kTileBytes);
+        tma_load_3d(sbase + kSmQ, &p.tmQ, 0, h, q0, B(kBarQ));
+        tma_load_3d(sbase + kSmQ + kBoxBytes, &p.tmQ, kBox, h, q0, B(kBarQ));
+      }
       int issued = 0;
       for (int j = 0; j < nt; ++j) {
-        const int s = j % kKV;
-        if (*s_abort || !mbar_wait_bounded(B(kBarKVFree + s), ((j / kKV) & 1) ^ 1)) {
+        const int s = j % ns;
+        if (*s_abort || !mbar_wait_bounded(free0 + 8u * s, ((j / ns) & 1) ^ 1)) {
           *s_abort = 1;
           break;
         }
         const int k0 = tile_at(tr, j) * kTile;
-        mbar_arrive_expect_tx(B(kBarKFull + s), kTileBytes);
-        tma_load_3d(sbase + kSmK + s * kTileBytes, &p.tmK, 0, h, k0, B(kBarKFull + s));
-        tma_load_3d(sbase + kSmK + s * kTileBytes + kBoxBytes, &p.tmK, kBox, h, k0, B(kBarKFull + s));
-        mbar_arrive_expect_tx(B(kBarVFull + s), kTileBytes);
-        tma_load_3d(sbase + kSmV + s * kTileBytes, &p.tmV, 0, h, k0, B(kBarVFull + s));
-        tma_load_3d(sbase + kSmV + s * kTileBytes + kBoxBytes, &p.tmV, kBox, h, k0, B(kBarVFull + s));
+        mbar_arrive_expect_tx(full0 + 8u * s, kTileBytes);
+        tma_load_3d(dst0 + s * kTileBytes, map, 0, h, k0, full0 + 8u * s);
+        tma_load_3d(dst0 + s * kTileBytes + kBoxBytes, map, kBox, h, k0, full0 + 8u * s);
         issued = j + 1;
       }
       // drain: every issued copy has landed before the CTA may exit
-      mbar_wait_bounded(B(kBarQ), 0);
-      for (int j = max(0, issued - kKV); j < issued; ++j) {
-        mbar_wait_bounded(B(kBarKFull + j % kKV), (j / kKV) & 1);
-        mbar_wait_bounded(B(kBarVFull + j % kKV), (j / kKV) & 1);
-      }
+      if (is_k) mbar_wait_bounded(B(kBarQ), 0);
+      for (int j = max(0, issued - ns); j < issued; ++j) mbar_wait_bounded(full0 + 8u * (j % ns), (j / ns) & 1);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
       bool ok = mbar_wait_bounded(B(kBarQ), 0);
-      const uint32_t aQ = sbase + kSmQ, aP = sbase + kSmP;
+      const uint32_t aQ = sbase + kSmQ;
       for (int j = 0; j <= nt && ok; ++j) {
-        if (j < nt) {  // S_j = Q K_j^T
-          const int s = j % kKV, sb = j & 1;
-          ok = !*s_abort && mbar_wait_bounded(B(kBarKFull + s), (j / kKV) & 1) &&
-               mbar_wait_bounded(B(kBarSFree + sb), ((j >> 1) & 1) ^ 1);
+        if (j < nt) {  // S_j = Q K_j^T, once the softmax has read S_{j-1}
+          const int s = j % kKS;
+          ok = !*s_abort && mbar_wait_bounded(B(kBarKFull + s), (j / kKS) & 1) &&
+               mbar_wait_bounded(B(kBarSFree), (j & 1) ^ 1);
           if (!ok) break;
           tc_fence_after();
           const uint32_t aK = sbase + kSmK + s * kTileBytes;
-          const uint32_t dS = tmem + (sb ? kColS1 : kColS0);
+          const uint32_t dS = tmem + kColS;
+          TC_CYC(j, 8);  // S_j issue
 #pragma unroll
           for (int kk = 0; kk < kD / 16; ++kk) {
             const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
             mma_bf16(dS, smem_desc(aQ + off, 16, 1024), smem_desc(aK + off, 16, 1024), kIdescQK, kk > 0);
           }
-          mma_commit(B(kBarSFull + sb));
+          mma_commit(B(kBarSFull));
+          mma_commit(B(kBarKFree + s));
         }
-        if (j >= 1) {  // O += P_{j-1} V_{j-1}
-          const int jp = j - 1, s = jp % kKV;
-          ok = !*s_abort && mbar_wait_bounded(B(kBarPFull), jp & 1) &&
-               mbar_wait_bounded(B(kBarVFull + s), (jp / kKV) & 1);
+        if (j >= 1) {  // O += P_{j-1} V_{j-1}, P from TMEM
+          const int jp = j - 1, s = jp % kVS, pb = jp & 1;
+          ok = !*s_abort && mbar_wait_bounded(B(kBarPFull + pb), (jp >> 1) & 1) &&
+               mbar_wait_bounded(B(kBarVFull + s), (jp / kVS) & 1);
           if (!ok) break;
+          TC_CYC(jp, 9);  // PV_jp issue (P and V ready)
           tc_fence_after();
           const uint32_t aV = sbase + kSmV + s * kTileBytes;
+          const uint32_t tP = tmem + (pb ? kColP1 : kColP0);
+          // 16 keys = 8 columns of bf16 pairs per step; keys 0..63 into O_A, 64..127 into O_B
 #pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk) {
-            const uint32_t offP = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-            mma_bf16(tmem + kColO, smem_desc(aP + offP, 16, 1024), smem_desc(aV + kk * 2048, kBoxBytes, 1024),
-                     kIdescPV, (jp > 0 || kk > 0));
-          }
-          mma_commit(B(kBarODone));
-          mma_commit(B(kBarKVFree + s));
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            mma_bf16_ta(tmem + (kk < 4 ? kColOA : kColOB), tP + kk * 8, smem_desc(aV + kk * 2048, kBoxBytes, 1024),
+                        kIdescPV, (jp > 0 || (kk & 3) > 0));
+          mma_commit(B(kBarPFree + pb));
+          mma_commit(B(kBarVFree + s));
         }
       }
       if (!ok) *s_abort = 1;
@@ -404,30 +453,31 @@ __global__ void __launch_bounds__(kThreads, 1) masked_tc_kernel(const __grid_con
     }
   } else {
     // ---------------------------------------------------------- softmax
-    const int hf = (warp - 2) >> 2;  // which part of the row: columns kHalf*hf ..
+    const int hf = (warp - 2) >> 2;  // which half of the row: keys kHalf*hf .. of each tile
     const int quarter = warp & 3;    // TMEM lanes 32*quarter .. +31
     const int r = quarter * 32 + lane;
     const int i = q0 + r;            // query row
     const int col0 = hf * kHalf;
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-    // this part of row r of P: box col0/64, first 16-byte chunk (col0 % 64)/8
-    uint8_t* Pbox = smem + kSmP + (col0 / kBox) * kBoxBytes + r * 128;
-    const int chunk0 = (col0 % kBox) / 8;
+    const uint32_t colO = hf ? kColOB : kColOA;  // this half's output accumulator
     float m_ref = -INFINITY, l_sum = 0.f;
     bool ok = true;
     for (int j = 0; j < nt; ++j) {
-      const int sb = j & 1;
       // After a timed-out wait a thread stops waiting but keeps arriving and
-      // joining the named barriers, so no thread of the CTA can be left
+      // joining the named barrier, so no thread of the CTA can be left
       // waiting on it; its rows are written as NaN.
-      if (ok && (*s_abort || !mbar_wait_bounded(B(kBarSFull + sb), (j >> 1) & 1))) ok = false;
+      const bool stamp = warp == 2 && lane == 0;
+      if (stamp) TC_CYC(j, 0);  // start waiting for S_j
+      if (ok && (*s_abort || !mbar_wait_bounded(B(kBarSFull), j & 1))) ok = false;
+      if (stamp) TC_CYC(j, 1);  // S_j ready
       tc_fence_after();
       float s[kHalf];
 #pragma unroll
-      for (int c = 0; c < kHalf; c += 32) tmem_ld32(lane_base + (sb ? kColS1 : kColS0) + col0 + c, s + c);
+      for (int c = 0; c < kHalf; c += 32) tmem_ld32(lane_base + kColS + col0 + c, s + c);
       tmem_wait_ld();
+      if (stamp) TC_CYC(j, 2);  // S loaded
       tc_fence_before();
-      mbar_arrive(B(kBarSFree + sb));
+      mbar_arrive(B(kBarSFree));
 
       const int k0 = tile_at(tr, j) * kTile;
       const bool full = (k0 + kTile - 1 < p.L_m) && (q0 >= p.L_m || k0 + kTile - 1 <= q0);
@@ -441,15 +491,10 @@ __global__ void __launch_bounds__(kThreads, 1) masked_tc_kernel(const __grid_con
           we = i - k0;
         }
       }
-      // row maximum: this half, then the other half's through shared memory
       const float mh = full ? half_max<true>(s, col0, ra, wb, we) : half_max<false>(s, col0, ra, wb, we);
-      rmax[(sb * kSplit + hf) * kTile + r] = mh;
-      named_barrier_sync(1, kSoftmaxThreads);
-      float mt = mh;
-#pragma unroll
-      for (int k = 0; k < kSplit; ++k) mt = fmaxf(mt, rmax[(sb * kSplit + k) * kTile + r]);
       // lazy rescale: only when the max (log2 units) grew by more than 8
-      const float mt_s = mt * p.scale_log2;
+      const float mt_s = mh * p.scale_log2;
+      if (stamp) TC_CYC(j, 3);  // maximum
       const bool grow = mt_s > m_ref + 8.f;
       const float m_new = grow ? mt_s : m_ref;
       const float corr = grow ? ex2(m_ref - m_new) : 1.f;  // 0 when m_ref was -inf
@@ -457,57 +502,64 @@ __global__ void __launch_bounds__(kThreads, 1) masked_tc_kernel(const __grid_con
       uint32_t pk[kHalf / 2];
       const float lt = full ? half_exp<true>(s, col0, ra, wb, we, p.scale_log2, msub, pk)
                             : half_exp<false>(s, col0, ra, wb, we, p.scale_log2, msub, pk);
-      // P buffer and O are free once PV_{j-1} has completed
-      if (j >= 1 && ok && !mbar_wait_bounded(B(kBarODone), (j - 1) & 1)) ok = false;
+      if (stamp) TC_CYC(j, 4);  // exponentials
+      // P buffer j&1 is free once the PV MMAs of tile j-2 have completed
+      const int pb = j & 1;
+      if (j >= 2 && ok && !mbar_wait_bounded(B(kBarPFree + pb), ((j >> 1) & 1) ^ 1)) ok = false;
       tc_fence_after();
-      // this part of the P row: kHalf bf16 in 16-byte chunks, 128B-swizzled
-#pragma unroll
-      for (int cc = 0; cc < kHalf / 8; ++cc) {
-        const uint4 w = make_uint4(pk[cc * 4 + 0], pk[cc * 4 + 1], pk[cc * 4 + 2], pk[cc * 4 + 3]);
-        *reinterpret_cast<uint4*>(Pbox + (((chunk0 + cc) ^ (r & 7)) * 16)) = w;
-      }
+      // this half of the P row: kHalf/2 columns of bf16 pairs (key 2c in the low half)
+      if (stamp) TC_CYC(j, 5);  // P buffer free
+      tmem_st_pairs(lane_base + (pb ? kColP1 : kColP0) + col0 / 2, pk);
       if (j >= 1 && __any_sync(0xffffffffu, grow)) {
+        // this half's O row is accumulated by the PV MMAs of tile j-1: wait for them
+        if (ok && !mbar_wait_bounded(B(kBarPFree + (pb ^ 1)), ((j - 1) >> 1) & 1)) ok = false;
+        tc_fence_after();
 #pragma unroll 1
-        for (int c = 0; c < kHalf; c += 16) {
+        for (int c = 0; c < kD; c += 16) {
           float o[16];
-          tmem_ld16(lane_base + kColO + col0 + c, o);
+          tmem_ld16(lane_base + colO + c, o);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 16; ++e) o[e] *= corr;
-          tmem_st16(lane_base + kColO + col0 + c, o);
+          tmem_st16(lane_base + colO + c, o);
         }
-        tmem_wait_st();
       }
+      tmem_wait_st();
+      if (stamp) TC_CYC(j, 6);  // P stored (and O rescaled)
       l_sum = l_sum * corr + lt;
       m_ref = m_new;
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // P visible to the tensor core
       tc_fence_before();
-      mbar_arrive(B(kBarPFull));
+      mbar_arrive(B(kBarPFull + pb));
     }
-    // epilogue: O / l to global memory, l summed over both halves
-    if (ok && nt > 0 && (*s_abort || !mbar_wait_bounded(B(kBarODone), (nt - 1) & 1))) ok = false;
+    // epilogue: combine the halves, O = (w_A O_A + w_B O_B) / (w_A l_A + w_B l_B);
+    // this thread writes output columns col0 .. col0 + kHalf
+    if (ok && nt > 0 && (*s_abort || !mbar_wait_bounded(B(kBarPFree + ((nt - 1) & 1)), ((nt - 1) >> 1) & 1)))
+      ok = false;
     tc_fence_after();
     if (!ok) *s_abort = 1;
-    lsum[hf * kTile + r] = l_sum;
+    mfin[hf * kTile + r] = m_ref;
+    lfin[hf * kTile + r] = l_sum;
     named_barrier_sync(1, kSoftmaxThreads);
-    float l_tot = 0.f;
-#pragma unroll
-    for (int k = 0; k < kSplit; ++k) l_tot += lsum[k * kTile + r];
-    const float inv = (ok && !*s_abort) ? 1.f / l_tot : __int_as_float(0x7fc00000);
+    const float mA = mfin[r], mB = mfin[kTile + r];
+    const float M = fmaxf(mA, mB);  // finite: every row sees at least one key
+    const float wA = ex2(mA - M), wB = ex2(mB - M);  // 0 for a half that saw no key
+    const float inv = (ok && !*s_abort) ? 1.f / (wA * lfin[r] + wB * lfin[kTile + r]) : __int_as_float(0x7fc00000);
+    const float aA = wA * inv, aB = wB * inv;
     __nv_bfloat16* orow = p.O + ((size_t)i * p.H + h) * kD + col0;
 #pragma unroll 1
-    for (int c = 0; c < kHalf; c += 32) {
-      float o[32];
-      tmem_ld32(lane_base + kColO + col0 + c, o);
+    for (int c = 0; c < kHalf; c += 16) {
+      float oa[16], ob[16];
+      tmem_ld16(lane_base + kColOA + col0 + c, oa);
+      tmem_ld16(lane_base + kColOB + col0 + c, ob);
       tmem_wait_ld();
       if (i < p.L) {
 #pragma unroll
-        for (int e = 0; e < 32; e += 8) {
+        for (int e = 0; e < 16; e += 8) {
           uint4 w;
-          w.x = pack_bf16x2(o[e] * inv, o[e + 1] * inv);
-          w.y = pack_bf16x2(o[e + 2] * inv, o[e + 3] * inv);
-          w.z = pack_bf16x2(o[e + 4] * inv, o[e + 5] * inv);
-          w.w = pack_bf16x2(o[e + 6] * inv, o[e + 7] * inv);
+          w.x = pack_bf16x2(oa[e] * aA + ob[e] * aB, oa[e + 1] * aA + ob[e + 1] * aB);
+          w.y = pack_bf16x2(oa[e + 2] * aA + ob[e + 2] * aB, oa[e + 3] * aA + ob[e + 3] * aB);
+          w.z = pack_bf16x2(oa[e + 4] * aA + ob[e + 4] * aB, oa[e + 5] * aA + ob[e + 5] * aB);
+          w.w = pack_bf16x2(oa[e + 6] * aA + ob[e + 6] * aB, oa[e + 7] * aA + ob[e + 7] * aB);
           *reinterpret_cast<uint4*>(orow + c + e) = w;
         }
       }
@@ -566,6 +618,7 @@ cudaError_t launch_masked_forward_tc(const MaskedParams& mp, cudaStream_t stream
   p.H = mp.H;
   p.n_qtiles = (mp.L + kTile - 1) / kTile;
   p.scale_log2 = mp.scale_log2;
+  p.timing = mp.timing;
   static bool configured[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
