@@ -124,27 +124,32 @@ def run_prefill(iters: int, warmup: int):
             "tflops": tf, "visible_pairs_per_head": pairs,
             "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
                          "frac": tf / peak, "peak_kind": f"{kind} dense bf16 (burst)",
-                         "traffic": None, "algorithmic_flops_per_launch": flops,
+                         "traffic": recorded_traffic("prefill", PREFILL_SOURCES, "prefill_traffic.json"),
+                         "algorithmic_flops_per_launch": flops,
                          "kernel": "rswa::tc::masked_tc_kernel"},
             "dense_causal_flops": dense_causal}
 
 
-def kernel_source_sha() -> str:
+DECODE_SOURCES = ("decode.cu", "common.cuh", "internal.h")
+PREFILL_SOURCES = ("masked_tc.cu", "common.cuh", "internal.h")
+
+
+def kernel_source_sha(files=DECODE_SOURCES) -> str:
     h = hashlib.sha256()
-    for f in ("decode.cu", "common.cuh", "internal.h"):
+    for f in files:
         with open(os.path.join(ROOT, "reference_sliding_window_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload: str):
+def recorded_traffic(workload: str, files=DECODE_SOURCES, record: str = "decode_traffic.json"):
     """DRAM bytes per launch from the committed ncu summary, if it was taken
     on the current kernel source for this workload; else None."""
     try:
-        with open(os.path.join(ROOT, "profiles", "decode_traffic.json")) as f:
+        with open(os.path.join(ROOT, "profiles", record)) as f:
             d = json.load(f)
         rec = d.get(workload)
-        if rec and rec.get("source_sha") == kernel_source_sha():
+        if rec and rec.get("source_sha") == kernel_source_sha(files):
             return float(rec["dram_bytes_per_launch"])
     except Exception:
         pass
