@@ -8,35 +8,33 @@
 //   j <= i  and  (i < L_m  or  j < L_m  or  j > i - n).
 //
 // Design (B200):
-// * One CTA per (128-query tile, head); the grid is ordered heaviest tile
-//   first so that the hardware block scheduler approximates longest-job-first.
-// * The key tiles a query tile needs are the reference tiles [0, ceil(L_m/128))
-//   plus the 2-3 tiles of its causal band; every other tile is fully masked
-//   and skipped.  Only tiles that are not fully visible are masked per element.
-// * Warp 0 lane 0 loads Q once and streams K tiles with TMA (128B-swizzled
-//   boxes of 128 rows x 64 columns) into a 3-stage ring whose stages free as
-//   soon as their QK^T MMA completes; warp 10 lane 0 streams V tiles into a
-//   2-stage ring freed by the PV MMAs.  Separate rings and producers keep a
-//   K load from waiting behind a V stage, so copies run two tiles ahead of
-//   the MMAs and their latency stays hidden.  Warp 1 owns the
-//   tensor memory (512 columns: S, O_A, O_B, P double-buffered) and one lane
-//   issues the MMAs: S_j = Q K_j^T into TMEM, then the PV products of tile
-//   j-1 with P read from TMEM, so the QK^T of tile j overlaps the softmax of
-//   tile j-1.  Keeping P in tensor memory leaves shared memory to the Q, K
-//   and V operands: at N = 128 an MMA with both operands in shared memory
-//   already takes all of its bandwidth.
-// * Warps 2..9 run the softmax, two threads per query row: warps w and w+4
-//   read the same TMEM lanes, one the keys 0..63 of each tile, the other the
-//   keys 64..127.  Each half keeps its own running maximum and sum and its
-//   own output accumulator (O_A += P[:, 0:64] V[0:64], O_B += P[:, 64:128]
-//   V[64:128]), so the halves never wait for each other inside the loop;
-//   the two are combined by the log-sum-exp rule once, at the end.  A thread
-//   forms p = 2^(s*scale*log2e - m), stores its half of P (bf16 pairs) into
-//   the tile's P buffer in TMEM, and rescales its O row only when its
-//   maximum grew by more than 2^8 since the last rescale (the stale maximum
-//   keeps every exponent <= 2^8, exact in float32).  So the softmax of tile
-//   j waits for the PV MMAs of tile j-1 only when it rescales; otherwise
-//   only for those of tile j-2 (the P buffer it reuses).
+// * One CTA per (pair of 128-query tiles, head), so every K/V tile loaded
+//   into shared memory serves 256 queries: half the key/value traffic per
+//   FLOP of one tile per CTA, whose delivery from L2 bounded it.  The grid
+//   is ordered heaviest pair first so that the hardware block scheduler
+//   approximates longest-job-first.
+// * The key tiles a pair needs are the reference tiles [0, ceil(L_m/128))
+//   plus the tiles of the pair's causal band; every other tile is fully
+//   masked and skipped.  Only tiles that are not fully visible to a query
+//   tile are masked per element.
+// * Warp 0 lane 0 loads both Q tiles, then streams K tiles with TMA
+//   (128B-swizzled boxes of 128 rows x 64 columns) into a 2-stage ring freed
+//   once both QK^T MMAs of a tile completed; warp 10 lane 0 streams V tiles
+//   into a 2-stage ring freed by the PV MMAs.  Warp 1 owns the tensor memory
+//   (512 columns: S_a, S_b, O_a, O_b) and one lane issues the MMAs.
+// * Warps 2-5 run the softmax of query tile a, warps 6-9 that of tile b, one
+//   thread per query row (TMEM lane): it reads its 128 scores with
+//   tcgen05.ld (two passes of 64 columns: maximum, then exponentials), forms
+//   p = 2^(s*scale*log2e - m), and writes P (bf16 pairs) over the first 64
+//   columns of its S with tcgen05.st.  The PV MMA reads P from TMEM.
+// * Issue order per key tile j: PV_a(j), S_a(j+1), PV_b(j), S_b(j+1).  While
+//   one group computes exponentials, the tensor core runs the other group's
+//   products, and vice versa.  S_g(j+1) overwrites P_g(j) only after PV_g(j)
+//   in the tensor core's issue order.
+// * O_g is rescaled in TMEM only when a row maximum grew by more than 2^8
+//   since the last rescale (the stale maximum keeps every exponent <= 2^8,
+//   exact in float32).  The commit that signals S_g(j) also covers
+//   PV_g(j-1), so the rescale needs no wait of its own.
 // * Every wait is bounded; on a timeout the kernel marks its rows with NaN,
 //   drains its copies and MMAs, frees its tensor memory and returns.
 
@@ -61,25 +59,25 @@ namespace tc {
 
 constexpr int kTile = 128;     // query and key tile
 constexpr int kD = 128;        // head dim
-constexpr int kSplit = 2;              // softmax threads per query row
-constexpr int kHalf = 128 / kSplit;    // columns per softmax thread
+constexpr int kQT = 2;         // query tiles per CTA
+constexpr int kHalf = 64;      // score columns per pass
 constexpr int kBox = 64;       // columns per 128B-swizzled box (bf16)
 constexpr int kBoxBytes = kTile * kBox * 2;      // 16 KB
 constexpr int kTileBytes = 2 * kBoxBytes;        // 32 KB: 128 rows x 128 cols
-constexpr int kKS = 3;                           // K ring stages
+constexpr int kKS = 2;                           // K ring stages
 constexpr int kVS = 2;                           // V ring stages
-constexpr int kSoftmaxThreads = 128 * kSplit;    // warps 2 .. 2 + 4*kSplit - 1
+constexpr int kSoftmaxThreads = 128 * kQT;       // warps 2 .. 9
 constexpr int kVWarp = 2 + kSoftmaxThreads / 32;  // V producer warp (after the softmax warps)
 constexpr int kThreads = 64 + kSoftmaxThreads + 32;  // K producer, MMA, softmax, V producer
 constexpr int kTmemCols = 512;
-constexpr uint32_t kColS = 0, kColOA = 128, kColOB = 256, kColP0 = 384, kColP1 = 448;  // P: bf16 pairs
+// TMEM columns of query tile g: S_g at 128*g (P_g, bf16 pairs, over its first 64), O_g at 256 + 128*g
+constexpr uint32_t kColS = 0, kColO = 256;
 
 // Shared memory map (offsets from a 1024-byte aligned base).
-constexpr int kSmQ = 0;
-constexpr int kSmK = kSmQ + kTileBytes;
+constexpr int kSmQ = 0;                          // kQT tiles
+constexpr int kSmK = kSmQ + kQT * kTileBytes;
 constexpr int kSmV = kSmK + kKS * kTileBytes;
-constexpr int kSmRed = kSmV + kVS * kTileBytes;  // float mfin[kSplit][128], lfin[kSplit][128]
-constexpr int kSmBar = kSmRed + 2 * kSplit * kTile * 4;
+constexpr int kSmBar = kSmV + kVS * kTileBytes;
 constexpr int kSmBytes = kSmBar + 256 + 1024;    // + slack for 1024-byte alignment
 
 // Instruction descriptor of tcgen05.mma kind::f16: bf16 A and B, float32 D,
@@ -241,8 +239,9 @@ struct TcParams {
   unsigned long long* timing;  // RSWA_TIMING builds: per-tile cycle stamps of CTA 0
 };
 
-// RSWA_TIMING builds record clock64 stamps of CTA 0 for its first 32 tiles:
-// slot [j][k], k < 8 by softmax warp 2 lane 0, k >= 8 by the MMA thread.
+// RSWA_TIMING builds record clock64 stamps of CTA 0 for its first 32 key
+// tiles: slot [j][k], k < 8 by softmax warp 2 lane 0 (query tile a), k >= 8
+// by the MMA thread.
 #ifdef RSWA_TIMING
 #define TC_CYC(j, k) \
   do { if (p.timing && blockIdx.x == 0 && (j) < 32) p.timing[(j) * 16 + (k)] = clock64(); } while (0)
@@ -250,13 +249,13 @@ struct TcParams {
 #define TC_CYC(j, k) do {} while (0)
 #endif
 
-// Key tiles of query tile at q0: [0, A) then [B0, B1] (B0 > A-1 or empty).
+// Key tiles of the query rows [q0, q0 + len): [0, A) then [B0, B1] (B0 > A-1 or empty).
 struct TileRange {
   int A, B0, B1;
 };
 
-__device__ __forceinline__ TileRange tile_range(int q0, int L, int L_m, int n) {
-  const int q_last = min(q0 + kTile, L) - 1;
+__device__ __forceinline__ TileRange tile_range(int q0, int len, int L, int L_m, int n) {
+  const int q_last = min(q0 + len, L) - 1;
   TileRange r;
   if (q_last < L_m) {  // all prefix rows: causal
     r.A = q_last / kTile + 1;
@@ -276,11 +275,11 @@ __device__ __forceinline__ int tile_at(const TileRange& r, int j) { return j < r
 
 // Barrier slots (8 bytes each).
 enum : int {
-  kBarQ = 0, kBarKFull = 1, kBarKFree = 4, kBarVFull = 7, kBarVFree = 9, kBarSFull = 11, kBarSFree = 12,
-  kBarPFull = 13, kBarPFree = 15, kBarFinal = 17, kSlotTmem = 18, kSlotAbort = 19
+  kBarQ = 0, kBarKFull = 1, kBarKFree = 3, kBarVFull = 5, kBarVFree = 7, kBarSFull = 9, kBarPFull = 11,
+  kBarODone = 13, kBarFinal = 15, kSlotTmem = 16, kSlotAbort = 17
 };
 
-// One thread's half row of an S tile (64 columns starting at col0):
+// 64 columns (starting at col0) of one thread's row of an S tile:
 // maximum of the visible scores.  FULL: every column visible; otherwise the
 // row's visible columns are [0, ra) and [wb, we] (the reference keys, causal
 // for a prefix row, and the output window).
@@ -297,7 +296,7 @@ __device__ __forceinline__ float half_max(const float* s, int col0, int ra, int 
   return fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
 }
 
-// Exponentials of the half row, packed to bf16 pairs; returns their sum.
+// Exponentials of those 64 columns, packed to bf16 pairs; returns their sum.
 template <bool FULL>
 __device__ __forceinline__ float half_exp(const float* s, int col0, int ra, int wb, int we, float sl2, float msub,
                                           uint32_t* pk) {
@@ -328,19 +327,18 @@ __global__ void __launch_bounds__(kThreads, 1) masked_tc_kernel(const __grid_con
   auto B = [&](int slot) { return bar0 + 8u * slot; };
   volatile uint32_t* s_tmem = reinterpret_cast<volatile uint32_t*>(&bars[kSlotTmem]);
   volatile int* s_abort = reinterpret_cast<volatile int*>(&bars[kSlotAbort]);
-  float* mfin = reinterpret_cast<float*>(smem + kSmRed);  // [half][row]: final maxima
-  float* lfin = mfin + kSplit * kTile;                     // [half][row]: final sums
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // heaviest tiles first: the tiles holding output rows, then prefix tiles
+  // heaviest pairs first: the pairs holding output rows, then prefix pairs
   // from the largest down
   const int h = blockIdx.x % p.H;
   const int rank = blockIdx.x / p.H;
-  const int t_s = p.L_m / kTile;  // tiles made only of prefix rows
-  const int qt = rank < p.n_qtiles - t_s ? t_s + rank : t_s - 1 - (rank - (p.n_qtiles - t_s));
-  const int q0 = qt * kTile;
-  const TileRange tr = tile_range(q0, p.L, p.L_m, p.n);
+  const int n_pairs = (p.n_qtiles + kQT - 1) / kQT;
+  const int t_s = p.L_m / (kQT * kTile);  // pairs made only of prefix rows
+  const int pr = rank < n_pairs - t_s ? t_s + rank : t_s - 1 - (rank - (n_pairs - t_s));
+  const int q0 = pr * kQT * kTile;
+  const TileRange tr = tile_range(q0, kQT * kTile, p.L, p.L_m, p.n);
   const int nt = tile_count(tr);
 
   if (threadIdx.x == 0) {
@@ -353,11 +351,10 @@ __global__ void __launch_bounds__(kThreads, 1) masked_tc_kernel(const __grid_con
       mbar_init(B(kBarVFull + s), 1);
       mbar_init(B(kBarVFree + s), 1);
     }
-    mbar_init(B(kBarSFull), 1);
-    mbar_init(B(kBarSFree), kSoftmaxThreads);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(B(kBarPFull + s), kSoftmaxThreads);
-      mbar_init(B(kBarPFree + s), 1);
+    for (int g = 0; g < kQT; ++g) {
+      mbar_init(B(kBarSFull + g), 1);
+      mbar_init(B(kBarPFull + g), 128);
+      mbar_init(B(kBarODone + g), 1);
     }
     mbar_init(B(kBarFinal), 1);
     *s_abort = 0;
@@ -376,7 +373,7 @@ __global__ void __launch_bounds__(kThreads, 1) masked_tc_kernel(const __grid_con
 
   if (warp == 0 || warp == kVWarp) {
     // ---------------------------------------------------------- producers
-    // warp 0: Q, then the K ring; warp kVWarp: the V ring
+    // warp 0: both Q tiles, then the K ring; warp kVWarp: the V ring
     if (lane == 0) {
       const bool is_k = warp == 0;
       const int ns = is_k ? kKS : kVS;
@@ -384,9 +381,11 @@ __global__ void __launch_bounds__(kThreads, 1) masked_tc_kernel(const __grid_con
       const uint32_t dst0 = sbase + (is_k ? kSmK : kSmV);
       const CUtensorMap* map = is_k ? &p.tmK : &p.tmV;
       if (is_k) {
-        mbar_arrive_expect_tx(B(kBarQ), kTileBytes);
-        tma_load_3d(sbase + kSmQ, &p.tmQ, 0, h, q0, B(kBarQ));
-        tma_load_3d(sbase + kSmQ + kBoxBytes, &p.tmQ, kBox, h, q0, B(kBarQ));
+        mbar_arrive_expect_tx(B(kBarQ), kQT * kTileBytes);
+        for (int g = 0; g < kQT; ++g) {
+          tma_load_3d(sbase + kSmQ + g * kTileBytes, &p.tmQ, 0, h, q0 + g * kTile, B(kBarQ));
+          tma_load_3d(sbase + kSmQ + g * kTileBytes + kBoxBytes, &p.tmQ, kBox, h, q0 + g * kTile, B(kBarQ));
+        }
       }
       int issued = 0;
       for (int j = 0; j < nt; ++j) {
@@ -408,42 +407,53 @@ __global__ void __launch_bounds__(kThreads, 1) masked_tc_kernel(const __grid_con
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      bool ok = mbar_wait_bounded(B(kBarQ), 0);
-      const uint32_t aQ = sbase + kSmQ;
-      for (int j = 0; j <= nt && ok; ++j) {
-        if (j < nt) {  // S_j = Q K_j^T, once the softmax has read S_{j-1}
-          const int s = j % kKS;
-          ok = !*s_abort && mbar_wait_bounded(B(kBarKFull + s), (j / kKS) & 1) &&
-               mbar_wait_bounded(B(kBarSFree), (j & 1) ^ 1);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t aK = sbase + kSmK + s * kTileBytes;
-          const uint32_t dS = tmem + kColS;
-          TC_CYC(j, 8);  // S_j issue
+      // S_g(j) = Q_g K_j^T into S_g
+      auto issue_s = [&](int g, int j) {
+        const uint32_t aQ = sbase + kSmQ + g * kTileBytes;
+        const uint32_t aK = sbase + kSmK + (j % kKS) * kTileBytes;
+        TC_CYC(j, 8 + g);
 #pragma unroll
-          for (int kk = 0; kk < kD / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-            mma_bf16(dS, smem_desc(aQ + off, 16, 1024), smem_desc(aK + off, 16, 1024), kIdescQK, kk > 0);
-          }
-          mma_commit(B(kBarSFull));
-          mma_commit(B(kBarKFree + s));
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
+          mma_bf16(tmem + kColS + 128 * g, smem_desc(aQ + off, 16, 1024), smem_desc(aK + off, 16, 1024), kIdescQK,
+                   kk > 0);
         }
-        if (j >= 1) {  // O += P_{j-1} V_{j-1}, P from TMEM
-          const int jp = j - 1, s = jp % kVS, pb = jp & 1;
-          ok = !*s_abort && mbar_wait_bounded(B(kBarPFull + pb), (jp >> 1) & 1) &&
-               mbar_wait_bounded(B(kBarVFull + s), (jp / kVS) & 1);
+        mma_commit(B(kBarSFull + g));
+      };
+      bool ok = mbar_wait_bounded(B(kBarQ), 0) && !*s_abort && mbar_wait_bounded(B(kBarKFull), 0);
+      if (ok) {
+        tc_fence_after();
+        for (int g = 0; g < kQT; ++g) issue_s(g, 0);
+        mma_commit(B(kBarKFree));
+      }
+      for (int j = 0; j < nt && ok; ++j) {
+        const int sv = j % kVS;
+        for (int g = 0; g < kQT; ++g) {
+          // O_g += P_g(j) V_j once group g has written P_g(j)
+          ok = !*s_abort && mbar_wait_bounded(B(kBarPFull + g), j & 1) &&
+               (g > 0 || mbar_wait_bounded(B(kBarVFull + sv), (j / kVS) & 1));
           if (!ok) break;
-          TC_CYC(jp, 9);  // PV_jp issue (P and V ready)
           tc_fence_after();
-          const uint32_t aV = sbase + kSmV + s * kTileBytes;
-          const uint32_t tP = tmem + (pb ? kColP1 : kColP0);
-          // 16 keys = 8 columns of bf16 pairs per step; keys 0..63 into O_A, 64..127 into O_B
+          TC_CYC(j, 10 + g);
+          const uint32_t aV = sbase + kSmV + sv * kTileBytes;
+          const uint32_t tP = tmem + kColS + 128 * g;
 #pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk)
-            mma_bf16_ta(tmem + (kk < 4 ? kColOA : kColOB), tP + kk * 8, smem_desc(aV + kk * 2048, kBoxBytes, 1024),
-                        kIdescPV, (jp > 0 || (kk & 3) > 0));
-          mma_commit(B(kBarPFree + pb));
-          mma_commit(B(kBarVFree + s));
+          for (int kk = 0; kk < kTile / 16; ++kk)  // 16 keys = 8 columns of bf16 pairs per step
+            mma_bf16_ta(tmem + kColO + 128 * g, tP + kk * 8, smem_desc(aV + kk * 2048, kBoxBytes, 1024), kIdescPV,
+                        (j > 0 || kk > 0));
+          if (g == kQT - 1) mma_commit(B(kBarVFree + sv));
+          if (j + 1 < nt) {
+            // S_g(j+1): issued after PV_g(j), which reads P_g(j) from the same columns
+            if (g == 0) {
+              ok = !*s_abort && mbar_wait_bounded(B(kBarKFull + (j + 1) % kKS), ((j + 1) / kKS) & 1);
+              if (!ok) break;
+              tc_fence_after();
+            }
+            issue_s(g, j + 1);
+            if (g == kQT - 1) mma_commit(B(kBarKFree + (j + 1) % kKS));
+          } else {
+            mma_commit(B(kBarODone + g));
+          }
         }
       }
       if (!ok) *s_abort = 1;
@@ -453,34 +463,25 @@ __global__ void __launch_bounds__(kThreads, 1) masked_tc_kernel(const __grid_con
     }
   } else {
     // ---------------------------------------------------------- softmax
-    const int hf = (warp - 2) >> 2;  // which half of the row: keys kHalf*hf .. of each tile
+    const int g = (warp - 2) >> 2;   // query tile of this group
     const int quarter = warp & 3;    // TMEM lanes 32*quarter .. +31
     const int r = quarter * 32 + lane;
-    const int i = q0 + r;            // query row
-    const int col0 = hf * kHalf;
+    const int q0g = q0 + g * kTile;
+    const int i = q0g + r;           // query row
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-    const uint32_t colO = hf ? kColOB : kColOA;  // this half's output accumulator
+    const uint32_t colS = kColS + 128 * g, colO = kColO + 128 * g;
+    const bool stamp = warp == 2 && lane == 0;
     float m_ref = -INFINITY, l_sum = 0.f;
     bool ok = true;
     for (int j = 0; j < nt; ++j) {
-      // After a timed-out wait a thread stops waiting but keeps arriving and
-      // joining the named barrier, so no thread of the CTA can be left
-      // waiting on it; its rows are written as NaN.
-      const bool stamp = warp == 2 && lane == 0;
-      if (stamp) TC_CYC(j, 0);  // start waiting for S_j
-      if (ok && (*s_abort || !mbar_wait_bounded(B(kBarSFull), j & 1))) ok = false;
-      if (stamp) TC_CYC(j, 1);  // S_j ready
+      // After a timed-out wait a thread stops waiting but keeps arriving, so
+      // the MMA thread is not left waiting on it; its rows are written as NaN.
+      if (stamp) TC_CYC(j, 0);
+      if (ok && (*s_abort || !mbar_wait_bounded(B(kBarSFull + g), j & 1))) ok = false;
+      if (stamp) TC_CYC(j, 1);
       tc_fence_after();
-      float s[kHalf];
-#pragma unroll
-      for (int c = 0; c < kHalf; c += 32) tmem_ld32(lane_base + kColS + col0 + c, s + c);
-      tmem_wait_ld();
-      if (stamp) TC_CYC(j, 2);  // S loaded
-      tc_fence_before();
-      mbar_arrive(B(kBarSFree));
-
       const int k0 = tile_at(tr, j) * kTile;
-      const bool full = (k0 + kTile - 1 < p.L_m) && (q0 >= p.L_m || k0 + kTile - 1 <= q0);
+      const bool full = (k0 + kTile - 1 < p.L_m) && (q0g >= p.L_m || k0 + kTile - 1 <= q0g);
       int ra = kTile, wb = 1, we = 0;
       if (!full) {
         if (i < p.L_m) {
@@ -491,29 +492,40 @@ __global__ void __launch_bounds__(kThreads, 1) masked_tc_kernel(const __grid_con
           we = i - k0;
         }
       }
-      const float mh = full ? half_max<true>(s, col0, ra, wb, we) : half_max<false>(s, col0, ra, wb, we);
+      // pass 1: row maximum over the 128 scores
+      float mh = -INFINITY;
+#pragma unroll 1
+      for (int c0 = 0; c0 < kTile; c0 += kHalf) {
+        float s[kHalf];
+        tmem_ld32(lane_base + colS + c0, s);
+        tmem_ld32(lane_base + colS + c0 + 32, s + 32);
+        tmem_wait_ld();
+        mh = fmaxf(mh, full ? half_max<true>(s, c0, ra, wb, we) : half_max<false>(s, c0, ra, wb, we));
+      }
+      if (stamp) TC_CYC(j, 2);
       // lazy rescale: only when the max (log2 units) grew by more than 8
       const float mt_s = mh * p.scale_log2;
-      if (stamp) TC_CYC(j, 3);  // maximum
       const bool grow = mt_s > m_ref + 8.f;
       const float m_new = grow ? mt_s : m_ref;
       const float corr = grow ? ex2(m_ref - m_new) : 1.f;  // 0 when m_ref was -inf
       const float msub = (m_new == -INFINITY) ? 0.f : m_new;
-      uint32_t pk[kHalf / 2];
-      const float lt = full ? half_exp<true>(s, col0, ra, wb, we, p.scale_log2, msub, pk)
-                            : half_exp<false>(s, col0, ra, wb, we, p.scale_log2, msub, pk);
-      if (stamp) TC_CYC(j, 4);  // exponentials
-      // P buffer j&1 is free once the PV MMAs of tile j-2 have completed
-      const int pb = j & 1;
-      if (j >= 2 && ok && !mbar_wait_bounded(B(kBarPFree + pb), ((j >> 1) & 1) ^ 1)) ok = false;
-      tc_fence_after();
-      // this half of the P row: kHalf/2 columns of bf16 pairs (key 2c in the low half)
-      if (stamp) TC_CYC(j, 5);  // P buffer free
-      tmem_st_pairs(lane_base + (pb ? kColP1 : kColP0) + col0 / 2, pk);
+      // pass 2: exponentials; P (bf16 pairs) goes over S columns [0, 64),
+      // which pass 2 has read by the time it writes them
+      float lt = 0.f;
+#pragma unroll 1
+      for (int c0 = 0; c0 < kTile; c0 += kHalf) {
+        float s[kHalf];
+        tmem_ld32(lane_base + colS + c0, s);
+        tmem_ld32(lane_base + colS + c0 + 32, s + 32);
+        tmem_wait_ld();
+        uint32_t pk[kHalf / 2];
+        lt += full ? half_exp<true>(s, c0, ra, wb, we, p.scale_log2, msub, pk)
+                   : half_exp<false>(s, c0, ra, wb, we, p.scale_log2, msub, pk);
+        tmem_st_pairs(lane_base + colS + c0 / 2, pk);
+      }
+      if (stamp) TC_CYC(j, 3);
+      // O_g was last written by PV_g(j-1), complete before S_g(j) was signalled
       if (j >= 1 && __any_sync(0xffffffffu, grow)) {
-        // this half's O row is accumulated by the PV MMAs of tile j-1: wait for them
-        if (ok && !mbar_wait_bounded(B(kBarPFree + (pb ^ 1)), ((j - 1) >> 1) & 1)) ok = false;
-        tc_fence_after();
 #pragma unroll 1
         for (int c = 0; c < kD; c += 16) {
           float o[16];
@@ -525,41 +537,31 @@ __global__ void __launch_bounds__(kThreads, 1) masked_tc_kernel(const __grid_con
         }
       }
       tmem_wait_st();
-      if (stamp) TC_CYC(j, 6);  // P stored (and O rescaled)
+      if (stamp) TC_CYC(j, 4);
       l_sum = l_sum * corr + lt;
       m_ref = m_new;
       tc_fence_before();
-      mbar_arrive(B(kBarPFull + pb));
+      mbar_arrive(B(kBarPFull + g));
     }
-    // epilogue: combine the halves, O = (w_A O_A + w_B O_B) / (w_A l_A + w_B l_B);
-    // this thread writes output columns col0 .. col0 + kHalf
-    if (ok && nt > 0 && (*s_abort || !mbar_wait_bounded(B(kBarPFree + ((nt - 1) & 1)), ((nt - 1) >> 1) & 1)))
-      ok = false;
+    // epilogue: O / l to global memory
+    if (ok && (*s_abort || !mbar_wait_bounded(B(kBarODone + g), 0))) ok = false;
     tc_fence_after();
     if (!ok) *s_abort = 1;
-    mfin[hf * kTile + r] = m_ref;
-    lfin[hf * kTile + r] = l_sum;
-    named_barrier_sync(1, kSoftmaxThreads);
-    const float mA = mfin[r], mB = mfin[kTile + r];
-    const float M = fmaxf(mA, mB);  // finite: every row sees at least one key
-    const float wA = ex2(mA - M), wB = ex2(mB - M);  // 0 for a half that saw no key
-    const float inv = (ok && !*s_abort) ? 1.f / (wA * lfin[r] + wB * lfin[kTile + r]) : __int_as_float(0x7fc00000);
-    const float aA = wA * inv, aB = wB * inv;
-    __nv_bfloat16* orow = p.O + ((size_t)i * p.H + h) * kD + col0;
+    const float inv = (ok && !*s_abort) ? 1.f / l_sum : __int_as_float(0x7fc00000);
+    __nv_bfloat16* orow = p.O + ((size_t)i * p.H + h) * kD;
 #pragma unroll 1
-    for (int c = 0; c < kHalf; c += 16) {
-      float oa[16], ob[16];
-      tmem_ld16(lane_base + kColOA + col0 + c, oa);
-      tmem_ld16(lane_base + kColOB + col0 + c, ob);
+    for (int c = 0; c < kD; c += 32) {
+      float o[32];
+      tmem_ld32(lane_base + colO + c, o);
       tmem_wait_ld();
       if (i < p.L) {
 #pragma unroll
-        for (int e = 0; e < 16; e += 8) {
+        for (int e = 0; e < 32; e += 8) {
           uint4 w;
-          w.x = pack_bf16x2(oa[e] * aA + ob[e] * aB, oa[e + 1] * aA + ob[e + 1] * aB);
-          w.y = pack_bf16x2(oa[e + 2] * aA + ob[e + 2] * aB, oa[e + 3] * aA + ob[e + 3] * aB);
-          w.z = pack_bf16x2(oa[e + 4] * aA + ob[e + 4] * aB, oa[e + 5] * aA + ob[e + 5] * aB);
-          w.w = pack_bf16x2(oa[e + 6] * aA + ob[e + 6] * aB, oa[e + 7] * aA + ob[e + 7] * aB);
+          w.x = pack_bf16x2(o[e] * inv, o[e + 1] * inv);
+          w.y = pack_bf16x2(o[e + 2] * inv, o[e + 3] * inv);
+          w.z = pack_bf16x2(o[e + 4] * inv, o[e + 5] * inv);
+          w.w = pack_bf16x2(o[e + 6] * inv, o[e + 7] * inv);
           *reinterpret_cast<uint4*>(orow + c + e) = w;
         }
       }
@@ -628,7 +630,7 @@ cudaError_t launch_masked_forward_tc(const MaskedParams& mp, cudaStream_t stream
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
-  masked_tc_kernel<<<p.n_qtiles * p.H, kThreads, kSmBytes, stream>>>(p);
+  masked_tc_kernel<<<(p.n_qtiles + kQT - 1) / kQT * p.H, kThreads, kSmBytes, stream>>>(p);
   return cudaGetLastError();
 }
 
