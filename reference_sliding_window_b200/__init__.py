@@ -32,7 +32,13 @@ def library_version() -> str:
     return _native.lib().rswa_version().decode()
 
 
+# The raw current-stream query avoids building a Stream object on every call.
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
 def _stream_ptr(device: torch.device) -> int:
+    if _raw_stream is not None:
+        return _raw_stream(device.index)
     return torch.cuda.current_stream(device).cuda_stream
 
 
@@ -70,6 +76,8 @@ class RSWA:
         if dev.index is None:
             dev = torch.device("cuda", torch.cuda.current_device())
         self.device = dev
+        self._dev_index = dev.index
+        self._vec_shape = torch.Size((batch, H, d))
         self.L_m_cap, self.n, self.H, self.d, self.batch = L_m_cap, n, H, d, batch
         self.dtype, self.mode, self.T_cap = dtype, mode, T_cap
         self.window = n if mode == MODE_RSWA else T_cap
@@ -89,6 +97,7 @@ class RSWA:
                               self.k_cache.data_ptr(), self.v_cache.data_ptr(),
                               self.workspace.data_ptr(), ws_bytes, self._stream))
         self._h = h
+        self._lib = L
 
     # -- plumbing
     def _sync_stream(self) -> None:
@@ -98,7 +107,10 @@ class RSWA:
             self._stream = s
 
     def _vec(self, name, t):
-        _check_tensor(name, t, (self.batch, self.H, self.d), self.dtype, self.device)
+        # fast path of _check_tensor on cached values; the slow one names the problem
+        if not (isinstance(t, torch.Tensor) and t.dtype == self.dtype and t.shape == self._vec_shape
+                and t.get_device() == self._dev_index and t.is_contiguous()):
+            _check_tensor(name, t, (self.batch, self.H, self.d), self.dtype, self.device)
 
     def close(self) -> None:
         if getattr(self, "_h", None):
@@ -136,7 +148,7 @@ class RSWA:
         o = torch.empty_like(q) if out is None else out
         self._vec("out", o)
         self._sync_stream()
-        check(_native.lib().rswa_decode(self._h, q.data_ptr(), o.data_ptr(), float(scale)))
+        check(self._lib.rswa_decode(self._h, q.data_ptr(), o.data_ptr(), float(scale)))
         return o
 
     def append_decode(self, k: torch.Tensor, v: torch.Tensor, q: torch.Tensor,
@@ -147,8 +159,8 @@ class RSWA:
         o = torch.empty_like(q) if out is None else out
         self._vec("out", o)
         self._sync_stream()
-        check(_native.lib().rswa_append_decode(self._h, k.data_ptr(), v.data_ptr(), q.data_ptr(),
-                                               o.data_ptr(), float(scale)))
+        check(self._lib.rswa_append_decode(self._h, k.data_ptr(), v.data_ptr(), q.data_ptr(),
+                                           o.data_ptr(), float(scale)))
         return o
 
     def cache_len(self) -> list:

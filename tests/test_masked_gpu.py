@@ -35,6 +35,13 @@ def _run(L, L_m, n, H, d, dtype, seed):
     (700, 300, 128, 2, 128, "bf16"),
     (520, 129, 1, 3, 128, "bf16"),
     (400, 255, 300, 2, 64, "bf16"),   # window wider than the outputs
+    # tensor-core kernel (bf16, d=128), which takes query tiles in pairs:
+    (128, 128, 16, 1, 128, "bf16"),   # one tile; its partner lies wholly past L
+    (1000, 513, 200, 2, 128, "bf16"), # ragged last pair
+    (768, 256, 64, 2, 128, "bf16"),   # L_m on a pair boundary
+    (640, 384, 5, 3, 128, "bf16"),    # L_m on a tile boundary inside a pair
+    (600, 600, 8, 2, 128, "bf16"),    # L_m = L: causal everywhere
+    (900, 100, 10000, 1, 128, "bf16"),  # window wider than the sequence: full causal
 ])
 def test_masked_forward_every_row(L, L_m, n, H, d, dtype):
     Q, K, V, O = _run(L, L_m, n, H, d, dtype, seed=L + n)
