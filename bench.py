@@ -96,6 +96,61 @@ def measured_tensor_peak():
         return FALLBACK_BF16_TFLOPS, "fallback"
 
 
+CURVE_T = (1, 32, 64, 128, 256, 512, 1024, 2048, 4096, 6144)
+
+
+def run_curve(w, lens, samples: int = 8):
+    """Per-step decode latency against the output length T, for the R-SWA
+    cache and for the same kernel over the full cache (every output kept):
+    the constant-cost curve against the growing one.  Each sample is one
+    fused append+decode launch, timed alone with CUDA events after an L2
+    flush; the median of `samples` consecutive steps is reported at each T."""
+    import torch
+    from reference_sliding_window_b200 import MODE_FULL, MODE_RSWA, RSWA, synth
+    dev = torch.device("cuda", torch.cuda.current_device())
+    B, H, d, n = w["B"], w["H"], w["d"], w["n"]
+    dt = synth.torch_dtype(w["dtype"])
+    s = 2 if w["dtype"] == "bf16" else 4
+    L_m_cap = max(lens)
+    T_top = CURVE_T[-1] + samples + 1
+    flush = torch.empty(2 * torch.cuda.get_device_properties(dev).L2_cache_size, dtype=torch.uint8, device=dev)
+    pool = synth.normal((16, 3, B, H, d), 4000, w["dtype"], "cuda")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    out = {"T": list(CURVE_T), "samples": samples, "timing": "isolated launches after an L2 flush, median"}
+    for name, mode in (("rswa", MODE_RSWA), ("full", MODE_FULL)):
+        a = RSWA(L_m_cap, n, H, d, B, dt, mode=mode, T_cap=T_top, device=dev)
+        Kr = synth.normal((B, H, L_m_cap, d), 4100, w["dtype"], "cuda")
+        Vr = synth.normal((B, H, L_m_cap, d), 4200, w["dtype"], "cuda")
+        a.load_reference(Kr, Vr, lens)
+        del Kr, Vr
+        o = torch.empty((B, H, d), dtype=dt, device=dev)
+        T, us, gbs = 0, [], []
+        for Tc in CURVE_T:
+            while T < Tc - 1:  # the next launch appends output Tc
+                x = pool[T % 16]
+                a.append_decode(x[0], x[1], x[2], out=o)
+                T += 1
+            ts = []
+            for _ in range(samples):
+                x = pool[T % 16]
+                flush.zero_()
+                e0.record()
+                a.append_decode(x[0], x[1], x[2], out=o)
+                e1.record()
+                e1.synchronize()
+                ts.append(e0.elapsed_time(e1) * 1e3)
+                T += 1
+            t_us = statistics.median(ts)
+            rows = sum((L + min(n, Tc)) if mode == MODE_RSWA else (L + Tc) for L in lens)
+            us.append(round(t_us, 2))
+            gbs.append(round(H * (2 * rows * d * s + 4 * B * d * s) / t_us / 1e3, 1))
+        a.check()
+        out[f"{name}_us"] = us
+        out[f"{name}_gbs"] = gbs
+        del a
+    return out
+
+
 def run_prefill(iters: int, warmup: int):
     """Times rswa_masked_forward on the 32K teacher-forced config (inputs
     252 MB, larger than L2).  Returns a dict for the JSON line."""
@@ -408,6 +463,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["prefill"], default="single_doc")
     ap.add_argument("--prefill-iters", type=int, default=10, help="timed masked-prefill calls (0: skip)")
+    ap.add_argument("--curve", type=int, default=1, help="1: add per-step latency vs T, R-SWA and full cache")
     ap.add_argument("--layers", type=int, default=0, help="layer caches cycled (0: 2 x L2 rule)")
     ap.add_argument("--e2e-steps", type=int, default=256)
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle timing")
@@ -458,6 +514,7 @@ def main():
             cpu = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample}
         value = whole_job_rate(res["tok_sum"], res["el_max"])
         prefill = run_prefill(args.prefill_iters, 3) if (args.prefill_iters > 0 and world == 1) else None
+        curve = run_curve(w, lens) if (args.curve and world == 1 and w["B"] * max(lens) <= 16384) else None
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": res["K"],
             "warmup": args.warmup, "ms_per_step": 1e3 * res["el_max"] / res["K"], "higher_is_better": True,
@@ -481,6 +538,7 @@ def main():
             "gpu_launches": res["launches"],
             "cpu_baseline": cpu,
             "prefill": prefill,
+            "vs_output_length": curve,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
