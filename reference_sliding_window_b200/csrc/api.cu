@@ -106,6 +106,8 @@ struct rswa_ctx {
   std::vector<int32_t> Lm;    // host copy of the reference lengths
   int plan_window;            // output rows the current plan covers
   int n_ctas;
+  int max_clusters;           // resident clusters of kDecodeCluster decode CTAs
+  bool cluster_plan;          // the current plan merges each slab inside one cluster
   std::vector<DecodeItem> items;
   std::vector<int32_t> cta_begin;
 };
@@ -124,11 +126,17 @@ static rswa_status use_device(rswa_ctx* c) {
   return RSWA_OK;
 }
 
-// Span planner: the planned rows of every (b, h) slab (b-major, then h) are
-// laid end to end in 32-row stages and cut into G nearly equal contiguous
-// spans, one per CTA, G = min(#SMs, #stages).  A span splits into items at
-// slab boundaries, so every CTA streams the same number of stages (+-1) and
-// a slab is merged from only as many partials as spans that touch it.
+// Two planners.
+// Cluster plan, when every slab can have a resident cluster of its own
+// (few slabs, e.g. one sequence): slab bh goes to the kDecodeCluster CTAs of
+// cluster bh, each taking a contiguous eighth of its 32-row stages, and the
+// cluster merges its partials in the leader's shared memory.
+// Span plan otherwise: the planned rows of every (b, h) slab (b-major, then
+// h) are laid end to end in 32-row stages and cut into G nearly equal
+// contiguous spans, one per CTA, G = min(#SMs, #stages).  A span splits
+// into items at slab boundaries, so every CTA streams the same number of
+// stages (+-1) and a slab is merged from only as many partials as spans
+// that touch it (through global memory and tickets).
 static void make_plan(rswa_ctx* c) {
   const int nbh = c->B * c->H;
   std::vector<int> rows(nbh), stages(nbh);
@@ -140,6 +148,32 @@ static void make_plan(rswa_ctx* c) {
       stages[b * c->H + h] = (r + 31) / 32;
       total += (r + 31) / 32;
     }
+  }
+  const int Gc = nbh * kDecodeCluster;
+  c->cluster_plan = nbh <= c->max_clusters && Gc <= c->lay.max_ctas && Gc <= c->lay.items_cap;
+  if (c->cluster_plan) {
+    c->items.clear();
+    c->cta_begin.assign(Gc + 1, 0);
+    for (int bh = 0; bh < nbh; ++bh) {
+      const int S = stages[bh];
+      for (int r = 0; r < kDecodeCluster; ++r) {
+        const int g = bh * kDecodeCluster + r;
+        const int st0 = (int)((long long)S * r / kDecodeCluster), st1 = (int)((long long)S * (r + 1) / kDecodeCluster);
+        DecodeItem it{};
+        it.bh = bh;
+        it.row0 = st0 * 32;
+        it.rows = std::max(0, std::min(rows[bh], st1 * 32) - it.row0);  // 0 when the slab has < 8 stages
+        it.part = g;
+        it.part_first = bh * kDecodeCluster;
+        it.nparts = kDecodeCluster;
+        it.last = (r == kDecodeCluster - 1) ? 1 : 0;
+        c->cta_begin[g] = g;
+        c->items.push_back(it);
+      }
+    }
+    c->cta_begin[Gc] = Gc;
+    c->n_ctas = Gc;
+    return;
   }
   const int G = (int)std::min<long long>(std::min(c->num_sms, c->lay.max_ctas), total);
   c->items.clear();
@@ -276,6 +310,8 @@ extern "C" rswa_status rswa_init(rswa_handle* out, rswa_mode mode, int L_m_cap, 
   c->T_host = 0;
   c->plan_window = 0;
   c->n_ctas = 0;
+  c->max_clusters = decode_max_active_clusters(dtype == RSWA_BF16 ? kBF16 : kF32, d);
+  c->cluster_plan = false;
   cudaError_t e = cudaMemsetAsync(c->ws, 0, lay.total, c->stream);
   if (e != cudaSuccess) {
     delete c;
@@ -418,6 +454,7 @@ static rswa_status run_decode(rswa_ctx* c, const void* k, const void* v, const v
   const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)c->d);
   p.scale_log2 = sc * 1.4426950408889634f;
   p.timing = g_timing;
+  p.cluster_merge = c->cluster_plan ? 1 : 0;
   // Only rswa_load_reference writes the reference rows, and its kernel
   // fences its writes before retiring, so every later decode may copy them
   // before its dependency wait.

@@ -94,7 +94,10 @@ struct DecTraits {
   static constexpr size_t kMetaOffset = (kRedOffset + kBatch * (2 * kW + kW * D) * 4 + 16 + 15) / 16 * 16;
   static constexpr size_t kLmOffset = kMetaOffset + sizeof(DecodeItem) * kPreItems;
   static constexpr size_t kQOffset = kLmOffset + 4 * kPreItems;
-  static constexpr size_t kSmemBytes = kQOffset + 4 * (size_t)kPreItems * D;
+  // cluster merge: the leader's mbarrier and partials[kDecodeCluster][D + 4]
+  static constexpr size_t kClBarOffset = (kQOffset + 4 * (size_t)kPreItems * D + 15) / 16 * 16;
+  static constexpr size_t kClBufOffset = kClBarOffset + 16;
+  static constexpr size_t kSmemBytes = kClBufOffset + 4 * (size_t)kDecodeCluster * (D + 4);
   // partials that fit in the stage ring when it doubles as merge buffer
   static constexpr int kMergeCap = (int)(kBarOffset / ((D + 4) * 4));
 };
@@ -133,6 +136,49 @@ __device__ __forceinline__ int atomic_add_relaxed(int32_t* p, int v) {
   int old;
   asm volatile("atom.relaxed.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
   return old;
+}
+
+// ---- thread-block cluster helpers (cluster-merge plan)
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Address of the same shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t cluster_map(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_remote_release(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+// Every thread of every CTA of the cluster (all threads must execute it).
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Bounded wait on a local mbarrier phase with cluster-scope acquire (the
+// arrivals came from other CTAs of the cluster).  Its limit is four times
+// the others': a CTA whose own waits timed out still arrives, about one
+// limit late, and the leader must outlive every store into its shared
+// memory.
+__device__ __forceinline__ bool mbar_wait_cluster_bounded(uint32_t bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (true) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    if (ok) return true;
+    if (clock64() - t0 > 4 * kWaitLimitCycles) return false;
+  }
 }
 
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
@@ -255,6 +301,8 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
   DecodeItem* s_items = reinterpret_cast<DecodeItem*>(smem + Tr::kMetaOffset);
   int* s_lm = reinterpret_cast<int*>(smem + Tr::kLmOffset);
   float* s_q = reinterpret_cast<float*>(smem + Tr::kQOffset);
+  const uint32_t cl_bar = smem_u32(smem + Tr::kClBarOffset);
+  float* cl_buf = reinterpret_cast<float*>(smem + Tr::kClBufOffset);  // [kDecodeCluster][D + 4]
   float* merge_buf = reinterpret_cast<float*>(smem);  // the stage ring, once drained
 
   const int warp = threadIdx.x >> 5;
@@ -267,6 +315,7 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
       mbar_init(smem_u32(&empty_bar[s]), 32 * Tr::kSplit);  // every lane of the owning group
     }
     *s_abort = 0;
+    if (p.cluster_merge) mbar_init(cl_bar, kDecodeCluster);  // one arrival per CTA of the cluster
     fence_barrier_init();
   }
   // The plan and the reference lengths are written by host copies ordered
@@ -284,6 +333,10 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
     s_lm[threadIdx.x] = p.Lm[item.bh / p.H];
   }
   __syncthreads();
+  // Cluster-merge plan: the leader's barrier must be initialised before any
+  // CTA of the cluster arrives on it.  Every thread passes here (no thread
+  // has exited yet), so this hardware barrier cannot be left waiting.
+  if (p.cluster_merge) cluster_sync_all();
   griddep_launch_dependents();
   auto item_at = [&](int it) -> DecodeItem {
     const int li = it - it_begin;
@@ -607,6 +660,14 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
       }
       if (item.nparts == 1) {
         store_elem(static_cast<T*>(p.o) + (size_t)item.bh * D + dd, acc / Ls);
+      } else if (p.cluster_merge) {
+        // this CTA's partial into slot `rank` of the cluster leader's buffer
+        const uint32_t slot = cluster_map(smem_u32(cl_buf + (size_t)cluster_rank() * (D + 4)), 0);
+        st_cluster_f32(slot + 4u * dd, acc);
+        if (dd == 0) {
+          st_cluster_f32(slot + 4u * D, M);
+          st_cluster_f32(slot + 4u * (D + 1), Ls);
+        }
       } else {
         float* P = p.partials + (size_t)item.part * (D + 4);
         P[dd] = acc;
@@ -618,6 +679,12 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
     }
     named_barrier_sync(1, NT);  // partials written; red_* are reused by the next batch
     if (tid == 0 && it0 == it_begin) RSWA_STAMP(10);
+    if (p.cluster_merge) {
+      // one item per CTA: arrive on the leader's barrier with release at
+      // cluster scope (after the barrier, so it covers every thread's stores)
+      if (tid == 0 && item_at(it0).nparts > 1) mbar_arrive_remote_release(cluster_map(cl_bar, 0));
+      continue;
+    }
     // Tickets of the batch's split items right away: one release fence
     // (after the barrier, so it covers every thread's partial writes), then
     // relaxed increments in flight together; their values are read at the end.
@@ -644,6 +711,25 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
   }
 
   if (tid == 0) RSWA_STAMP(4);
+  // ---- cluster-merge plan: the leader folds the cluster's partials
+  if (p.cluster_merge && it_end > it_begin && cluster_rank() == 0 && item_at(it_begin).nparts > 1 && tid < D) {
+    const DecodeItem item = item_at(it_begin);
+    const bool ok = mbar_wait_cluster_bounded(cl_bar, 0);
+    if (!ok && tid == 0) flag_error(p.err, kErrWaitTimeout);
+    if (ok) {
+      float M = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < kDecodeCluster; ++i) M = fmaxf(M, cl_buf[i * (D + 4) + D]);  // finite: the slab has rows
+      float acc = 0.f, L = 0.f;
+#pragma unroll
+      for (int i = 0; i < kDecodeCluster; ++i) {
+        const float w = exp2f(cl_buf[i * (D + 4) + D] - M);  // exp2(-inf) = 0 for an empty part
+        acc = fmaf(w, cl_buf[i * (D + 4) + tid], acc);
+        L = fmaf(w, cl_buf[i * (D + 4) + D + 1], L);
+      }
+      store_elem(static_cast<T*>(p.o) + (size_t)item.bh * D + tid, acc / L);
+    }
+  }
   // ---- split items: the CTA holding the last ticket of a slab merges it.
   if (tid == 0) {
     int l0 = 0, l1 = 0;
@@ -705,12 +791,49 @@ static cudaError_t launch_one(const DecodeParams& p, int grid, cudaStream_t stre
   cfg.blockDim = dim3(Tr::kThreads);
   cfg.dynamicSmemBytes = Tr::kSmemBytes;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = p.cluster_merge ? kDecodeCluster : 1;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = p.cluster_merge ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, decode_kernel<T, D, A>, p);
+}
+
+template <typename T, int D>
+static int max_clusters(void) {
+  using Tr = DecTraits<T, D>;
+  if (cudaFuncSetAttribute(decode_kernel<T, D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)Tr::kSmemBytes) != cudaSuccess)
+    return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(kDecodeCluster);
+  cfg.blockDim = dim3(Tr::kThreads);
+  cfg.dynamicSmemBytes = Tr::kSmemBytes;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kDecodeCluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_kernel<T, D, A>, p);
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, decode_kernel<T, D, true>, &cfg) != cudaSuccess) {
+    cudaGetLastError();  // clear the sticky-free error so later calls are unaffected
+    return 0;
+  }
+  return n;
+}
+
+int decode_max_active_clusters(int elem, int D) {
+  if (elem == kBF16 && D == 128) return max_clusters<__nv_bfloat16, 128>();
+  if (elem == kBF16 && D == 64) return max_clusters<__nv_bfloat16, 64>();
+  if (elem == kF32 && D == 128) return max_clusters<float, 128>();
+  if (elem == kF32 && D == 64) return max_clusters<float, 64>();
+  return 0;
 }
 
 template <typename T, int D>

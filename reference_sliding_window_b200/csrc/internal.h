@@ -75,11 +75,18 @@ struct DecodeParams {
   int32_t* done;
   int32_t* err;
   int ref_stable;        // 1: the reference rows are final (see decode.cu); 0: read after the wait
+  int cluster_merge;     // 1: the kDecodeCluster CTAs of a slab form a cluster and merge in
+                         //    the leader's shared memory (one item per CTA)
   float scale_log2;      // softmax scale * log2(e)
   unsigned long long* timing;  // profiling stamps (RSWA_TIMING builds), may be null
 };
 
 // Launch the split-K decode kernel (append: fused ring write + T advance).
+// CTAs per cluster in the cluster-merge plan.
+constexpr int kDecodeCluster = 8;
+// Clusters of kDecodeCluster decode CTAs that can be resident at once (0 on error).
+int decode_max_active_clusters(int elem, int D);
+
 cudaError_t launch_decode(int elem, int D, bool append, const DecodeParams& p, int grid,
                           cudaStream_t stream);
 // Dynamic shared memory the decode kernel needs for (elem, D).
