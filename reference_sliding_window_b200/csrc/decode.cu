@@ -51,6 +51,8 @@
 #include <math.h>
 #include <stdio.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -136,6 +138,19 @@ __device__ __forceinline__ int atomic_add_relaxed(int32_t* p, int v) {
   int old;
   asm volatile("atom.relaxed.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
   return old;
+}
+
+// acc + a.lo*b.lo + a.hi*b.hi for two packed bf16 pairs, with fp32
+// accumulation (each bf16 product is exact in fp32).
+__device__ __forceinline__ float fma2_bf16(uint32_t a, uint32_t b, float acc) {
+  asm("{.reg .b16 al, ah, bl, bh;\n\t"
+      "mov.b32 {al, ah}, %1;\n\t"
+      "mov.b32 {bl, bh}, %2;\n\t"
+      "fma.rn.f32.bf16 %0, al, bl, %0;\n\t"
+      "fma.rn.f32.bf16 %0, ah, bh, %0;\n\t}"
+      : "+f"(acc)
+      : "r"(a), "r"(b));
+  return acc;
 }
 
 // ---- thread-block cluster helpers (cluster-merge plan)
@@ -286,6 +301,9 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
   using Tr = DecTraits<T, D>;
   constexpr int EPV = Tr::kEPV, LPR = Tr::kLPR, RPI = Tr::kRPI, NS = Tr::kStages, NV = Tr::kNV;
   constexpr int kStageRows = Tr::kStageRows, WR = Tr::kWarpRows, GR = Tr::kGroups;
+  // bf16: q.k from the packed words with mixed-precision FMAs (q unscaled,
+  // the scale applied to the finished score); fp32: unpacked, q scaled.
+  constexpr bool kMixed = std::is_same<T, __nv_bfloat16>::value;
   constexpr int W = Tr::kW, NT = Tr::kConsumerThreads;
   constexpr int RB = Tr::kRowBytes, SB = Tr::kStageBytes;
 
@@ -449,10 +467,14 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
       const int i = x / VPR, v = x % VPR;
       const uint4 qu =
           *reinterpret_cast<const uint4*>(static_cast<const T*>(p.q) + (size_t)s_items[i].bh * D + v * EPV);
-      float f[EPV];
-      Vec16<T>::unpack(qu, f);
+      if (kMixed) {
+        reinterpret_cast<uint4*>(s_q + i * D)[v] = qu;  // raw bf16
+      } else {
+        float f[EPV];
+        Vec16<T>::unpack(qu, f);
 #pragma unroll
-      for (int e = 0; e < EPV; ++e) s_q[i * D + v * EPV + e] = f[e] * p.scale_log2;
+        for (int e = 0; e < EPV; ++e) s_q[i * D + v * EPV + e] = f[e] * p.scale_log2;
+      }
     }
   }
   named_barrier_sync(1, NT);
@@ -502,7 +524,11 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
     }
 
     float qf[EPV], of[EPV];
-    if (li < kPreItems) {
+    uint4 qraw = make_uint4(0, 0, 0, 0);
+    if (kMixed) {
+      qraw = li < kPreItems ? reinterpret_cast<const uint4*>(s_q + li * D)[sub]
+                            : *reinterpret_cast<const uint4*>(static_cast<const T*>(p.q) + (size_t)item.bh * D + sub * EPV);
+    } else if (li < kPreItems) {
 #pragma unroll
       for (int e = 0; e < EPV; e += 4) {
         const float4 q4 = *reinterpret_cast<const float4*>(s_q + li * D + sub * EPV + e);
@@ -562,11 +588,18 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
             *reinterpret_cast<uint4*>(static_cast<T*>(p.vc_w) + c_off) = vsub;
             sub_k = k;
           }
-          float f[EPV];
-          Vec16<T>::unpack(u, f);
           float acc = 0.f;
+          if (kMixed) {
+            acc = fma2_bf16(qraw.x, u.x, acc);
+            acc = fma2_bf16(qraw.y, u.y, acc);
+            acc = fma2_bf16(qraw.z, u.z, acc);
+            acc = fma2_bf16(qraw.w, u.w, acc);
+          } else {
+            float f[EPV];
+            Vec16<T>::unpack(u, f);
 #pragma unroll
-          for (int e = 0; e < EPV; ++e) acc = fmaf(qf[e], f[e], acc);
+            for (int e = 0; e < EPV; ++e) acc = fmaf(qf[e], f[e], acc);
+          }
           part[k] = acc;
         }
         if (gs == 0 && lane == 0) RSWA_CYC(3);
@@ -590,7 +623,7 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
         const bool valid = my_row < nr;
         const bool owner = sub < NV;  // one lane per row adds to the sum
         if (gs == 0 && lane == 0) RSWA_CYC(4);
-        const float sc = valid ? part[0] : -INFINITY;
+        const float sc = valid ? (kMixed ? part[0] * p.scale_log2 : part[0]) : -INFINITY;
         float mx = sc;
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
