@@ -10,14 +10,22 @@
 // depend on storage order, so ring rows can be read in slot order.
 //
 // Design (B200):
-// * The planned rows of all (b, h) slabs are laid end to end and cut into
-//   one contiguous span per CTA (one persistent CTA per SM), in 32-row
-//   stages; a span splits into items at slab boundaries, so only the first
-//   and last item of a CTA can be part of a slab shared with another CTA.
-// * One producer lane streams the planned K and V stages of its span into a
-//   ring of shared-memory buffers with bulk async copies (cp.async.bulk,
-//   completion on mbarriers).  It needs no device state, so the first copy
-//   is issued right after the plan is read.
+// * Two launch plans (made on the host).  Span plan: the planned rows of all
+//   (b, h) slabs are laid end to end and cut into one contiguous span per
+//   CTA (one persistent CTA per SM), in 32-row stages; a span splits into
+//   items at slab boundaries, so only the first and last item of a CTA can
+//   be part of a slab shared with another CTA.  Cluster plan, when every
+//   slab can have a resident cluster of its own: slab bh goes to the
+//   kDecodeCluster CTAs of cluster bh, one contiguous part each.
+// * Before waiting on the previous kernel (programmatic dependent launch):
+//   barrier set-up, the plan and reference lengths (host-written) staged in
+//   shared memory, copies of the leading stages made only of reference rows
+//   (written only by the reference load, whose kernel fences before it
+//   retires), and an L2 prefetch of the remaining rows.  The ring rows, q
+//   and the step counter are read after the wait.  The next kernel may
+//   launch as soon as this one has started.
+// * One producer lane streams the stages into a ring of shared-memory
+//   buffers with bulk async copies (cp.async.bulk, completion on mbarriers).
 // * Stage g (32 rows, counted over the launch) goes to consumer warp group
 //   g % kGroups and ring buffer g % kStages; the kSplit warps of a group
 //   each take kWarpRows rows of it.  kStages is a multiple of kGroups, so a
@@ -26,27 +34,29 @@
 //   unambiguous.
 // * A warp's part of a stage is NV = 8 warp-wide 16-byte loads of K (and of
 //   V): 16 rows of bf16 d=128.  The warp reads it from shared memory (one
-//   row = LPR lanes), forms NV partial dot products per lane and reduces
-//   them with a transposed butterfly over NV lanes plus plain shuffles over
-//   the rest of the row's lanes (NV-1 + log2(LPR/NV) shuffles leave every
-//   lane one finished score), then updates a float32 online softmax (base-2
-//   exponent with the scale folded into q) and its slice of the output.
-//   Rows at or past the current cache length are masked.  Splitting stages
-//   over warps keeps the serial work of one warp short (at small cache
-//   sizes the launch is latency-bound) while the copies stay 8 KB each.
-// * Warps merge per item in shared memory.  Items of a shared slab leave a
-//   partial (m, l, o); at the end of its span a CTA takes one acq_rel ticket
-//   per such item and the last CTA of a slab merges its partials with the
-//   log-sum-exp rule (one round of independent loads).  Nothing spins.
+//   row = LPR lanes), forms NV partial dot products per lane (bf16:
+//   mixed-precision FMAs on the packed words) and reduces them with a
+//   transposed butterfly over NV lanes plus plain shuffles over the rest of
+//   the row's lanes (NV-1 + log2(LPR/NV) shuffles leave every lane one
+//   finished score), then updates a float32 online softmax (base 2) and its
+//   slice of the output.  Rows at or past the current cache length are
+//   masked.  Splitting stages over warps keeps the serial work of one warp
+//   short (at small cache sizes the launch is latency-bound) while the
+//   copies stay 8 KB each.
+// * Warps merge per batch of items in shared memory.  Items of a shared
+//   slab leave a partial (m, l, o).  Span plan: one release fence and a
+//   relaxed ticket per split item; the CTA holding a slab's last ticket
+//   acquires and merges the slab's partials with the log-sum-exp rule (one
+//   round of independent loads).  Cluster plan: each CTA stores its partial
+//   into the leader CTA's shared memory and arrives on the leader's
+//   mbarrier (release, cluster scope); the leader waits and merges.
 // * APPEND: the consumer that meets the slot row substitutes the new k/v
 //   (the staged copy of that row may predate the write) and stores them into
 //   the slot.  Each CTA reads the step counter T once and then takes a
 //   launch ticket; the CTA with the last ticket knows every CTA has read T
 //   and advances it.  One kernel per decode step, replayable in a CUDA graph.
-// * Programmatic dependent launch: barrier set-up, the plan reads and an L2
-//   prefetch of the rows to stream happen before waiting on the previous
-//   kernel of the stream (the plan is host-written; L2 is coherent), and the
-//   next kernel may launch as soon as this one has started.
+// * Every wait is bounded; a timeout sets the device error word and the
+//   kernel finishes without trapping.
 
 #include <math.h>
 #include <stdio.h>
