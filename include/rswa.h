@@ -107,6 +107,10 @@ size_t rswa_workspace_bytes(int L_m_cap, int window_cap, int H, int d, int batch
  *     (stream-ordered).
  *   n: window size (RSWA mode, >= 1).  T_cap: max outputs (FULL mode, >= 1).
  *   The other of n / T_cap is ignored.
+ *   Decode plan: when every (b, h) slab can have a resident cluster of
+ *   8 CTAs, a slab's partial results are merged inside its cluster;
+ *   otherwise across CTAs through the workspace.  The environment variable
+ *   RSWA_DECODE_PLAN=span, read here, forces the second plan.
  * Requires a CUDA device of compute capability 10.0 (B200). */
 rswa_status rswa_init(rswa_handle* out, rswa_mode mode, int L_m_cap, int n, int T_cap,
                       int H, int d, int batch, rswa_dtype dtype,

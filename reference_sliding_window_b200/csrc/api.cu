@@ -7,6 +7,7 @@
 #include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <algorithm>
@@ -311,6 +312,8 @@ extern "C" rswa_status rswa_init(rswa_handle* out, rswa_mode mode, int L_m_cap, 
   c->plan_window = 0;
   c->n_ctas = 0;
   c->max_clusters = decode_max_active_clusters(dtype == RSWA_BF16 ? kBF16 : kF32, d);
+  const char* plan = getenv("RSWA_DECODE_PLAN");  // "span": never use the cluster plan
+  if (plan && strcmp(plan, "span") == 0) c->max_clusters = 0;
   c->cluster_plan = false;
   cudaError_t e = cudaMemsetAsync(c->ws, 0, lay.total, c->stream);
   if (e != cudaSuccess) {

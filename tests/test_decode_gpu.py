@@ -20,6 +20,17 @@ def _cuda():
         pytest.skip("needs a CUDA device")
 
 
+@pytest.fixture(params=["auto", "span"])
+def plan(request, monkeypatch):
+    """Both decode plans: the library's choice (the cluster merge for these
+    few-slab cases) and the span plan with its merge across CTAs."""
+    if request.param == "span":
+        monkeypatch.setenv("RSWA_DECODE_PLAN", "span")
+    else:
+        monkeypatch.delenv("RSWA_DECODE_PLAN", raising=False)
+    return request.param
+
+
 # ------------------------------------------------------------ index parity
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
@@ -94,7 +105,7 @@ def test_decode_before_any_output_sees_reference_only():
     ("bf16", 128, 33, [257, 31, 96, 128], True),
     ("f32", 64, 5, [500], True),
 ])
-def test_small_shapes_every_step(dtype, d, n, ref_lens, fused):
+def test_small_shapes_every_step(dtype, d, n, ref_lens, fused, plan):
     T = 3 * n + 5
     case = synth.decode_case(B=len(ref_lens), H=2, d=d, ref_lens=ref_lens, n=n, T=T, dtype=dtype, seed=5 + n)
     a = make_attn(case)
@@ -120,7 +131,7 @@ def test_full_mode_and_its_capacity():
     a.check()
 
 
-def test_full_mode_replans_past_first_window():
+def test_full_mode_replans_past_first_window(plan):
     # FULL mode plans 64 output rows at a time; cross several boundaries.
     case = synth.decode_case(B=1, H=2, d=64, ref_lens=[30], n=8, T=530, dtype="f32", seed=8)
     a = make_attn(case, mode=MODE_FULL, T_cap=600)
@@ -154,7 +165,7 @@ def test_state_errors():
 
 # ------------------------------------------------------------- CUDA graphs
 
-def test_graph_replay_advances_the_ring():
+def test_graph_replay_advances_the_ring(plan):
     """One captured append+decode replayed step after step: the device step
     counter and slot index make the graph reusable."""
     case = synth.decode_case(B=2, H=2, d=128, ref_lens=[300, 45], n=16, T=60, dtype="bf16", seed=11)
@@ -191,7 +202,7 @@ def _device_case(B, H, d, ref_lens, n, T, seed):
                              seed=seed, device="cuda")
 
 
-def test_single_document_full_size_sampled():
+def test_single_document_full_size_sampled(plan):
     """Batch 1, 10 heads, d=128, L_m=2592 (10 pages x 256 + 32 prompt),
     n=128, T=6144 steps, bf16: outputs sampled across the run."""
     case = _device_case(1, 10, 128, [2592], 128, 6144, 12)
