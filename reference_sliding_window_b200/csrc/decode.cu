@@ -71,7 +71,7 @@ namespace rswa {
 constexpr int kStageBudget = 192 * 1024;
 constexpr long long kPrefetchBytes = 256 * 1024;  // per CTA and per K/V tensor
 constexpr int kPrefetchChunk = 32 * 1024;
-// Items per CTA whose descriptor, reference length and (scaled) query are
+// Items per CTA whose descriptor, reference length and query (raw for bf16, scaled for fp32) are
 // staged in shared memory by the prologue; later items of a longer span
 // read them from global memory when they start.
 constexpr int kPreItems = 8;
