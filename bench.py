@@ -170,6 +170,15 @@ def run_prefill(iters: int, warmup: int):
     e1.record()
     torch.cuda.synchronize(dev)
     sec = e0.elapsed_time(e1) / 1e3 / iters
+    # ablation: the same tensors with no reference segment (L_m = 0, the
+    # plain sliding window of n the pages contrast R-SWA with)
+    e0.record()
+    for _ in range(iters):
+        masked_forward(Q, K, V, L_m=0, n=w["n"], out=O)
+    e1.record()
+    torch.cuda.synchronize(dev)
+    sec_swa = e0.elapsed_time(e1) / 1e3 / iters
+    pairs_swa = visible_pairs(w["L"], 0, w["n"])
     pairs = visible_pairs(w["L"], w["L_m"], w["n"])
     flops = 4.0 * w["d"] * pairs * w["H"]
     dense_causal = 4.0 * w["d"] * (w["L"] * (w["L"] + 1) // 2) * w["H"]
@@ -182,7 +191,9 @@ def run_prefill(iters: int, warmup: int):
                          "traffic": recorded_traffic("prefill", PREFILL_SOURCES, "prefill_traffic.json"),
                          "algorithmic_flops_per_launch": flops,
                          "kernel": "rswa::tc::masked_tc_kernel"},
-            "dense_causal_flops": dense_causal}
+            "dense_causal_flops": dense_causal,
+            "window_only_ablation": {"L_m": 0, "ms_per_call": sec_swa * 1e3, "visible_pairs_per_head": pairs_swa,
+                                     "tflops": 4.0 * w["d"] * pairs_swa * w["H"] / sec_swa / 1e12}}
 
 
 DECODE_SOURCES = ("decode.cu", "common.cuh", "internal.h")

@@ -178,13 +178,29 @@ void rswa_destroy(rswa_handle h);
  * visible from query p and -inf elsewhere:
  *   p <= L_m : j <= p                       (causal inside the prefix)
  *   p >  L_m : j <= L_m, or p-n+1 <= j <= p  (Eq.(1)-(2) with t = p-L_m+1)
- * Q, K, V, O: device [L][H][d] (token-major).  1 <= L_m <= L, n >= 1.
+ * Q, K, V, O: device [L][H][d] (token-major).  0 <= L_m <= L, n >= 1.
+ * L_m = 0 leaves no reference segment: every query sees p-n+1 .. p, the
+ * plain sliding window the pages contrast R-SWA with ("vanilla SWA",
+ * 核心导读 Fig. 1 and 方法展开 §1), for ablation.
  * BF16 runs on the tcgen05 tensor-core kernel (d = 128), F32 on a SIMT
  * kernel (d = 64 or 128).  Tiles the mask fully hides are skipped.
  * ---------------------------------------------------------------------- */
 rswa_status rswa_masked_forward(const void* Q, const void* K, const void* V, void* O,
                                 int L, int L_m, int n, int H, int d, rswa_dtype dtype,
                                 float scale, void* stream);
+
+/* Flags of rswa_masked_forward_ex. */
+typedef enum {
+  /* Every prefix query p <= L_m sees all reference keys 1..L_m (the pages
+   * are silent on prefix queries; without the flag they are causal). */
+  RSWA_FLAG_BIDIR_PREFIX = 1
+} rswa_forward_flags;
+
+/* rswa_masked_forward with flags (a bitwise OR of rswa_forward_flags; 0
+ * gives rswa_masked_forward).  Unknown flag bits return RSWA_ERR_ARG. */
+rswa_status rswa_masked_forward_ex(const void* Q, const void* K, const void* V, void* O,
+                                   int L, int L_m, int n, int H, int d, rswa_dtype dtype,
+                                   float scale, int flags, void* stream);
 
 /* ------------------------------------------------------------------------
  * Decode without allocation.  The pages have no counterpart to this call;

@@ -39,6 +39,12 @@ R4  Multi-head attention with H query heads = H key/value heads; heads are
 R5  Decode after T appends: the query of the newest output T produces
     output T+1 and sees N(T+1) = P ∪ outputs max(1, T+1-n) .. T, which is
     L_m + min(n, T) rows, Eq.(6).
+R6  L_m = 0 in the packed form leaves no reference segment: every query p
+    sees max(1, p-n+1) .. p, the plain sliding window the pages contrast
+    R-SWA with ([UOW-1] 核心导读 Fig. 1 and 方法展开 §1, "vanilla SWA").
+R7  Bidirectional prefix (an option; the pages are silent and R2 is the
+    default): every prefix query p <= L_m sees all of P = 1..L_m; outputs
+    are unchanged.
 """
 
 from __future__ import annotations
@@ -53,6 +59,7 @@ __all__ = [
     "window_positions",
     "visible_positions",
     "packed_visible_positions",
+    "bidir_prefix_visible_positions",
     "packed_mask",
     "attend",
     "masked_forward",
@@ -107,11 +114,20 @@ def packed_visible_positions(p: int, L_m: int, n: int) -> np.ndarray:
     return visible_positions(p - L_m + 1, L_m, n)
 
 
-def packed_mask(L: int, L_m: int, n: int) -> np.ndarray:
+def bidir_prefix_visible_positions(p: int, L_m: int, n: int) -> np.ndarray:
+    """As ``packed_visible_positions`` with a bidirectional prefix (reading
+    R7): a prefix query p <= L_m sees all of P."""
+    if 1 <= p <= L_m:
+        return reference_positions(L_m)
+    return packed_visible_positions(p, L_m, n)
+
+
+def packed_mask(L: int, L_m: int, n: int, bidir_prefix: bool = False) -> np.ndarray:
     """Explicit boolean mask M[p-1, j-1] = (j visible from query p), shape [L, L]."""
+    vis = bidir_prefix_visible_positions if bidir_prefix else packed_visible_positions
     M = np.zeros((L, L), dtype=bool)
     for p in range(1, L + 1):
-        M[p - 1, packed_visible_positions(p, L_m, n) - 1] = True
+        M[p - 1, vis(p, L_m, n) - 1] = True
     return M
 
 
@@ -234,7 +250,7 @@ def _default_scale(d: int, scale) -> float:
 
 
 def masked_forward(Q: np.ndarray, K: np.ndarray, V: np.ndarray, L_m: int, n: int,
-                   scale=None) -> np.ndarray:
+                   scale=None, bidir_prefix: bool = False) -> np.ndarray:
     """Teacher-forced form: O = softmax(Q K^T * scale + M) V per head with the
     explicit mask M of ``packed_mask`` (-inf where not visible).
     Q, K, V: [L, H, d]  ->  O: [L, H, d] float64."""
@@ -243,7 +259,7 @@ def masked_forward(Q: np.ndarray, K: np.ndarray, V: np.ndarray, L_m: int, n: int
     V = np.asarray(V, dtype=np.float64)
     L, H, d = Q.shape
     sc = _default_scale(d, scale)
-    M = packed_mask(L, L_m, n)
+    M = packed_mask(L, L_m, n, bidir_prefix)
     O = np.empty((L, H, d), dtype=np.float64)
     for h in range(H):
         S = (Q[:, h, :] @ K[:, h, :].T) * sc
@@ -256,14 +272,14 @@ def masked_forward(Q: np.ndarray, K: np.ndarray, V: np.ndarray, L_m: int, n: int
 
 
 def masked_forward_rows(Q: np.ndarray, K: np.ndarray, V: np.ndarray, L_m: int, n: int,
-                        rows: Sequence[int], scale=None) -> np.ndarray:
+                        rows: Sequence[int], scale=None, bidir_prefix: bool = False) -> np.ndarray:
     """Same as ``masked_forward`` for the selected 0-based query rows only
     (for sequences too long for the full [L, L] mask).  -> [len(rows), H, d]."""
     L, H, d = Q.shape
     sc = _default_scale(d, scale)
     out = np.empty((len(rows), H, d), dtype=np.float64)
     for i, r in enumerate(rows):
-        vis = packed_visible_positions(int(r) + 1, L_m, n) - 1
+        vis = (bidir_prefix_visible_positions if bidir_prefix else packed_visible_positions)(int(r) + 1, L_m, n) - 1
         for h in range(H):
             out[i, h] = attend(Q[r, h], K[vis, h], V[vis, h], sc)
     return out

@@ -194,8 +194,11 @@ class RSWA:
 
 
 def masked_forward(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, L_m: int, n: int,
-                   scale: float = 0.0, out: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """Teacher-forced R-SWA attention.  Q, K, V, out: [L, H, d] on a B200."""
+                   scale: float = 0.0, out: Optional[torch.Tensor] = None,
+                   bidir_prefix: bool = False) -> torch.Tensor:
+    """Teacher-forced R-SWA attention.  Q, K, V, out: [L, H, d] on a B200.
+    L_m = 0: no reference segment (the plain sliding window of n).
+    bidir_prefix: prefix queries see every reference key (default: causal)."""
     if Q.dim() != 3:
         raise ValueError("Q must be [L, H, d]")
     L, H, d = Q.shape
@@ -207,7 +210,8 @@ def masked_forward(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, L_m: int, 
     O = torch.empty_like(Q) if out is None else out
     _check_tensor("out", O, (L, H, d), Q.dtype, Q.device)
     with torch.cuda.device(Q.device):
-        check(_native.lib().rswa_masked_forward(Q.data_ptr(), K.data_ptr(), V.data_ptr(), O.data_ptr(),
-                                                L, int(L_m), int(n), H, d, _DT[Q.dtype], float(scale),
-                                                _stream_ptr(Q.device)))
+        check(_native.lib().rswa_masked_forward_ex(Q.data_ptr(), K.data_ptr(), V.data_ptr(), O.data_ptr(),
+                                                   L, int(L_m), int(n), H, d, _DT[Q.dtype], float(scale),
+                                                   _native.FLAG_BIDIR_PREFIX if bidir_prefix else 0,
+                                                   _stream_ptr(Q.device)))
     return O

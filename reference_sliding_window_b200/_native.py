@@ -14,9 +14,10 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librswa.so"
 OK, ERR_ARG, ERR_STATE, ERR_CAPACITY, ERR_UNSUPPORTED, ERR_CUDA, ERR_DEVICE = range(7)
 STATUS_NAMES = ["RSWA_OK", "RSWA_ERR_ARG", "RSWA_ERR_STATE", "RSWA_ERR_CAPACITY",
                 "RSWA_ERR_UNSUPPORTED", "RSWA_ERR_CUDA", "RSWA_ERR_DEVICE"]
-# rswa_dtype / rswa_mode
+# rswa_dtype / rswa_mode / rswa_forward_flags
 F32, BF16 = 0, 1
 MODE_RSWA, MODE_FULL = 0, 1
+FLAG_BIDIR_PREFIX = 1
 
 _i, _f, _p, _sz = C.c_int, C.c_float, C.c_void_p, C.c_size_t
 _PROTOS = {
@@ -35,6 +36,7 @@ _PROTOS = {
     "rswa_check": (_i, [_p]),
     "rswa_destroy": (None, [_p]),
     "rswa_masked_forward": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _p]),
+    "rswa_masked_forward_ex": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _i, _p]),
     "rswa_decode_noalloc": (_i, [_p, _p, _i, C.POINTER(C.c_int32), _p, _p, _i, _i, _i, _i, _f, _p]),
     "rswa_last_error": (C.c_char_p, []),
     "rswa_version": (C.c_char_p, []),

@@ -580,13 +580,20 @@ extern "C" rswa_status rswa_check(rswa_handle h) {
 extern "C" rswa_status rswa_masked_forward(const void* Q, const void* K, const void* V, void* O, int L,
                                            int L_m, int n, int H, int d, rswa_dtype dtype, float scale,
                                            void* stream) {
+  return rswa_masked_forward_ex(Q, K, V, O, L, L_m, n, H, d, dtype, scale, 0, stream);
+}
+
+extern "C" rswa_status rswa_masked_forward_ex(const void* Q, const void* K, const void* V, void* O, int L,
+                                              int L_m, int n, int H, int d, rswa_dtype dtype, float scale,
+                                              int flags, void* stream) {
   if (!Q || !K || !V || !O) return fail(RSWA_ERR_ARG, "rswa_masked_forward: null tensor");
+  if (flags & ~(int)RSWA_FLAG_BIDIR_PREFIX) return fail(RSWA_ERR_ARG, "rswa_masked_forward: unknown flags %d", flags);
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
     return fail(RSWA_ERR_ARG, "rswa_masked_forward: tensors must be 16-byte aligned");
   if (!dtype_ok(dtype)) return fail(RSWA_ERR_UNSUPPORTED, "rswa_masked_forward: unknown dtype");
   if (d != 64 && d != 128) return fail(RSWA_ERR_UNSUPPORTED, "rswa_masked_forward: head dim %d", d);
   if (L < 1 || H < 1) return fail(RSWA_ERR_ARG, "rswa_masked_forward: L=%d H=%d", L, H);
-  if (L_m < 1 || L_m > L) return fail(RSWA_ERR_ARG, "rswa_masked_forward: L_m=%d outside [1, L=%d]", L_m, L);
+  if (L_m < 0 || L_m > L) return fail(RSWA_ERR_ARG, "rswa_masked_forward: L_m=%d outside [0, L=%d]", L_m, L);
   if (n < 1) return fail(RSWA_ERR_ARG, "rswa_masked_forward: n=%d must be >= 1", n);
   if (!(scale == scale) || isinf(scale)) return fail(RSWA_ERR_ARG, "rswa_masked_forward: scale not finite");
   if ((long long)L * H * d >= (1ll << 31))
@@ -610,6 +617,7 @@ extern "C" rswa_status rswa_masked_forward(const void* Q, const void* K, const v
   p.D = d;
   const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)d);
   p.scale_log2 = sc * 1.4426950408889634f;
+  p.bidir_prefix = (flags & RSWA_FLAG_BIDIR_PREFIX) ? 1 : 0;
   p.timing = g_timing;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (dtype == RSWA_BF16 && d == 128) {

@@ -121,6 +121,7 @@ struct MaskedParams {
   void* O;
   int L, L_m, n, H, D;
   float scale_log2;
+  int bidir_prefix;             // 1: prefix queries see every reference key
   unsigned long long* timing;  // profiling stamps (RSWA_TIMING builds), may be null
 };
 // Sets the thread-local message returned by rswa_last_error().

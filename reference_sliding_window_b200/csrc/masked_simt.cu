@@ -4,8 +4,9 @@
 // Mask ("Unlimited OCR Works：一篇读懂 R-SWA 如何把长文档 OCR 从 for-loop 推向
 // one-shot", 方法展开 §3, Eq.(1)-(2)): the query at 1-based position p
 // produces output t = p - L_m + 1 and sees the reference rows 1..L_m plus
-// max(L_m+1, p-n+1)..p; a prefix query (p <= L_m) sees 1..p.  So each row
-// visits at most two contiguous key ranges and never tests a mask element.
+// max(L_m+1, p-n+1)..p; a prefix query (p <= L_m) sees 1..p (1..L_m with a
+// bidirectional prefix).  So each row visits at most two contiguous key
+// ranges and never tests a mask element.  L_m = 0 leaves the window alone.
 
 #include <math.h>
 
@@ -38,7 +39,7 @@ masked_simt_kernel(const __grid_constant__ MaskedParams p) {
   const int pos = row + 1;
   int r0b = 0, r0e, r1b = 0, r1e = 0;
   if (pos <= p.L_m) {
-    r0e = pos;
+    r0e = p.bidir_prefix ? p.L_m : pos;
   } else {
     r0e = p.L_m;
     r1b = max(p.L_m, pos - p.n);

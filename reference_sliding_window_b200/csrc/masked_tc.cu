@@ -235,6 +235,7 @@ struct TcParams {
   CUtensorMap tmQ, tmK, tmV;  // 3-D maps {d, H, L} of bf16, 64x1x128 boxes, 128B swizzle
   __nv_bfloat16* O;
   int L, L_m, n, H, n_qtiles;
+  int bidir;                  // 1: prefix queries see every reference key
   float scale_log2;
   unsigned long long* timing;  // RSWA_TIMING builds: per-tile cycle stamps of CTA 0
 };
@@ -254,11 +255,11 @@ struct TileRange {
   int A, B0, B1;
 };
 
-__device__ __forceinline__ TileRange tile_range(int q0, int len, int L, int L_m, int n) {
+__device__ __forceinline__ TileRange tile_range(int q0, int len, int L, int L_m, int n, bool bidir) {
   const int q_last = min(q0 + len, L) - 1;
   TileRange r;
-  if (q_last < L_m) {  // all prefix rows: causal
-    r.A = q_last / kTile + 1;
+  if (q_last < L_m) {  // all prefix rows: causal, or every reference key (bidirectional)
+    r.A = bidir ? (L_m + kTile - 1) / kTile : q_last / kTile + 1;
     r.B0 = 1;
     r.B1 = 0;
     return r;
@@ -338,7 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1) masked_tc_kernel(const __grid_con
   const int t_s = p.L_m / (kQT * kTile);  // pairs made only of prefix rows
   const int pr = rank < n_pairs - t_s ? t_s + rank : t_s - 1 - (rank - (n_pairs - t_s));
   const int q0 = pr * kQT * kTile;
-  const TileRange tr = tile_range(q0, kQT * kTile, p.L, p.L_m, p.n);
+  const TileRange tr = tile_range(q0, kQT * kTile, p.L, p.L_m, p.n, p.bidir != 0);
   const int nt = tile_count(tr);
 
   if (threadIdx.x == 0) {
@@ -481,11 +482,11 @@ __global__ void __launch_bounds__(kThreads, 1) masked_tc_kernel(const __grid_con
       if (stamp) TC_CYC(j, 1);
       tc_fence_after();
       const int k0 = tile_at(tr, j) * kTile;
-      const bool full = (k0 + kTile - 1 < p.L_m) && (q0g >= p.L_m || k0 + kTile - 1 <= q0g);
+      const bool full = (k0 + kTile - 1 < p.L_m) && (p.bidir || q0g >= p.L_m || k0 + kTile - 1 <= q0g);
       int ra = kTile, wb = 1, we = 0;
       if (!full) {
         if (i < p.L_m) {
-          ra = i + 1 - k0;
+          ra = (p.bidir ? p.L_m : i + 1) - k0;
         } else {
           ra = p.L_m - k0;
           wb = max(p.L_m, i - p.n + 1) - k0;
@@ -620,6 +621,7 @@ cudaError_t launch_masked_forward_tc(const MaskedParams& mp, cudaStream_t stream
   p.H = mp.H;
   p.n_qtiles = (mp.L + kTile - 1) / kTile;
   p.scale_log2 = mp.scale_log2;
+  p.bidir = mp.bidir_prefix;
   p.timing = mp.timing;
   static bool configured[64] = {false};
   int dev = 0;

@@ -67,6 +67,34 @@ def pin_packed_mask_small(o):
     assert got.shape == want.shape and (got == want).all(), got.astype(int)
 
 
+def pin_swa_mask_small(o):
+    # L_m = 0: no reference segment, the plain sliding window (reading R6).
+    want = np.array(_rows("swa_mask_L6_n2.txt"), dtype=bool)
+    got = o.packed_mask(6, 0, 2)
+    assert got.shape == want.shape and (got == want).all(), got.astype(int)
+
+
+def pin_bidir_prefix_mask_small(o):
+    want = np.array(_rows("packed_mask_bidir_L6_Lm3_n2.txt"), dtype=bool)
+    got = o.packed_mask(6, 3, 2, bidir_prefix=True)
+    assert got.shape == want.shape and (got == want).all(), got.astype(int)
+
+
+def pin_swa_and_bidir_predicates(o):
+    # Brute-force predicates, written independently of the set construction.
+    for n, L in ((1, 5), (2, 9), (3, 14), (7, 11), (20, 12)):
+        M = o.packed_mask(L, 0, n)
+        for p in range(1, L + 1):
+            for j in range(1, L + 1):
+                assert bool(M[p - 1, j - 1]) == (p - n < j <= p), (n, p, j)
+    for L_m, n, L in ((3, 2, 9), (1, 1, 6), (5, 3, 14), (6, 8, 10)):
+        M = o.packed_mask(L, L_m, n, bidir_prefix=True)
+        for p in range(1, L + 1):
+            for j in range(1, L + 1):
+                want = (j <= L_m) if p <= L_m else (j <= p and (j <= L_m or j > p - n))
+                assert bool(M[p - 1, j - 1]) == want, (L_m, n, p, j)
+
+
 def pin_cache_sizes(o):
     for L_m, n, T, c_mha, c_rswa, num, den in _rows("eq5_eq7_cache_sizes.txt"):
         assert o.occupancy_full(T, L_m) == c_mha
@@ -129,6 +157,53 @@ def pin_short_output_is_causal(o):
         ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=True)
         ref = ref.permute(1, 0, 2).numpy()
         assert np.allclose(got, ref, rtol=1e-12, atol=1e-12), np.abs(got - ref).max()
+
+
+def pin_swa_wide_window_is_causal(o):
+    # L_m = 0 and n >= L: the window covers every earlier token, so the form
+    # is plain causal attention (torch's fp64 SDPA as the library routine).
+    for L, n, H, d in ((17, 17, 2, 5), (9, 40, 1, 3)):
+        Q, K, V = _rand((L, H, d), 31), _rand((L, H, d), 32), _rand((L, H, d), 33)
+        got = o.masked_forward(Q, K, V, 0, n)
+        tq, tk, tv = (torch.from_numpy(x).permute(1, 0, 2) for x in (Q, K, V))
+        ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=True)
+        ref = ref.permute(1, 0, 2).numpy()
+        assert np.allclose(got, ref, rtol=1e-12, atol=1e-12), np.abs(got - ref).max()
+
+
+def pin_bidir_prefix_rows_are_full_attention(o):
+    # Bidirectional prefix: prefix rows are plain (non-causal) attention over
+    # the prefix block (torch's fp64 SDPA); output rows are those of the
+    # default form.
+    L, L_m, n, H, d = 15, 6, 3, 2, 4
+    Q, K, V = _rand((L, H, d), 34), _rand((L, H, d), 35), _rand((L, H, d), 36)
+    got = o.masked_forward(Q, K, V, L_m, n, bidir_prefix=True)
+    tq, tk, tv = (torch.from_numpy(x[:L_m]).permute(1, 0, 2) for x in (Q, K, V))
+    ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=False).permute(1, 0, 2).numpy()
+    assert np.allclose(got[:L_m], ref, rtol=1e-12, atol=1e-12), np.abs(got[:L_m] - ref).max()
+    base = o.masked_forward(Q, K, V, L_m, n)
+    assert np.allclose(got[L_m:], base[L_m:], rtol=0, atol=0)
+    rows = [0, L_m - 1, L_m, L - 1]
+    sub = o.masked_forward_rows(Q, K, V, L_m, n, rows, bidir_prefix=True)
+    assert np.allclose(sub, got[rows], rtol=1e-13, atol=1e-13)
+
+
+def pin_swa_brute_force(o):
+    # Scalar loops, math.exp, explicit window predicate; L_m = 0, tiny sizes.
+    L, n, H, d = 8, 3, 2, 3
+    Q, K, V = _rand((L, H, d), 37), _rand((L, H, d), 38), _rand((L, H, d), 39)
+    got = o.masked_forward(Q, K, V, 0, n)
+    scale = 1.0 / math.sqrt(d)
+    for h in range(H):
+        for p in range(1, L + 1):
+            vis = [j for j in range(1, L + 1) if p - n < j <= p]
+            s = {j: sum(Q[p - 1, h, c] * K[j - 1, h, c] for c in range(d)) * scale for j in vis}
+            mx = max(s.values())
+            w = {j: math.exp(s[j] - mx) for j in vis}
+            z = sum(w.values())
+            for c in range(d):
+                want = sum(w[j] * V[j - 1, h, c] for j in vis) / z
+                assert abs(got[p - 1, h, c] - want) < 1e-12, (h, p, c)
 
 
 def pin_identical_keys_mean(o):

@@ -106,11 +106,20 @@ def test_masked_forward_rejects_bad_arguments_before_device(lib):
     assert mf(None, p, p, p, 8, 2, 2, 1, 64, _native.F32, 0.0, None) == _native.ERR_ARG
     assert mf(p, p, p, p + 4, 8, 2, 2, 1, 64, _native.F32, 0.0, None) == _native.ERR_ARG
     assert mf(p, p, p, p, 8, 2, 2, 1, 80, _native.F32, 0.0, None) == _native.ERR_UNSUPPORTED
-    assert mf(p, p, p, p, 8, 0, 2, 1, 64, _native.F32, 0.0, None) == _native.ERR_ARG
+    assert mf(p, p, p, p, 8, -1, 2, 1, 64, _native.F32, 0.0, None) == _native.ERR_ARG  # L_m = 0 is the plain window
     assert mf(p, p, p, p, 8, 9, 2, 1, 64, _native.F32, 0.0, None) == _native.ERR_ARG
     assert mf(p, p, p, p, 8, 2, 0, 1, 64, _native.F32, 0.0, None) == _native.ERR_ARG
     assert mf(p, p, p, p, 8, 2, 2, 1, 64, _native.F32, float("nan"), None) == _native.ERR_ARG
     assert mf(p, p, p, p, 8, 2, 2, 1, 64, 3, 0.0, None) == _native.ERR_UNSUPPORTED
+
+
+def test_masked_forward_ex_rejects_unknown_flags(lib):
+    buf = C.create_string_buffer(256)
+    p = (C.cast(buf, C.c_void_p).value + 15) // 16 * 16
+    mfx = lib.rswa_masked_forward_ex
+    assert mfx(p, p, p, p, 8, 2, 2, 1, 64, _native.F32, 0.0, 2, None) == _native.ERR_ARG
+    assert mfx(p, p, p, p, 8, 2, 2, 1, 64, _native.F32, 0.0, -1, None) == _native.ERR_ARG
+    assert mfx(None, p, p, p, 8, 2, 2, 1, 64, _native.F32, 0.0, _native.FLAG_BIDIR_PREFIX, None) == _native.ERR_ARG
 
 
 def test_product_path_has_no_oracle_dependency():

@@ -49,6 +49,27 @@ def test_masked_forward_every_row(L, L_m, n, H, d, dtype):
     assert_close(O, want, dtype, "masked forward")
 
 
+@pytest.mark.parametrize("L,L_m,n,H,d,dtype,bidir", [
+    # L_m = 0: no reference segment, the plain sliding window
+    (300, 0, 16, 2, 64, "f32", False),
+    (700, 0, 128, 2, 128, "bf16", False),
+    (520, 0, 1, 2, 128, "bf16", False),
+    (257, 0, 300, 1, 128, "f32", False),
+    # bidirectional prefix
+    (300, 100, 16, 2, 64, "f32", True),
+    (700, 300, 128, 2, 128, "bf16", True),
+    (640, 384, 5, 2, 128, "bf16", True),   # L_m on a tile boundary inside a pair
+    (200, 200, 8, 1, 128, "bf16", True),   # all prefix: full attention
+])
+def test_masked_forward_window_and_prefix_options(L, L_m, n, H, d, dtype, bidir):
+    Q, K, V = synth.prefill_case(L, H, d, dtype, seed=L + n + 7)
+    O = masked_forward(Q.cuda(), K.cuda(), V.cuda(), L_m=L_m, n=n, bidir_prefix=bidir)
+    torch.cuda.synchronize()
+    want = oracle.masked_forward(Q.double().numpy(), K.double().numpy(), V.double().numpy(), L_m, n,
+                                 bidir_prefix=bidir)
+    assert_close(O, want, dtype, "masked forward options")
+
+
 def test_teacher_forced_full_size_sampled_rows():
     """Packed 32768-token sequence, 10 heads, d=128, L_m=12832 reference
     tokens + 19936 outputs with n=128, bf16: boundary rows plus random rows."""

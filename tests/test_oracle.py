@@ -122,10 +122,32 @@ def _mut_decode_window(m):
     m.decode_visible_positions = lambda T, L_m, n: orig(max(T, 1), L_m, n)
 
 
+def _mut_swa_keeps_first_token(m):
+    # the window forgets that there is no reference segment: key 1 stays visible
+    orig = m.packed_visible_positions
+
+    def packed_visible_positions(p, L_m, n):
+        vis = orig(p, L_m, n)
+        return np.union1d(vis, [1]) if L_m == 0 else vis
+    m.packed_visible_positions = packed_visible_positions
+
+
+def _mut_bidir_stays_causal(m):
+    m.bidir_prefix_visible_positions = lambda p, L_m, n: m.packed_visible_positions(p, L_m, n)
+
+
+def _mut_bidir_sees_outputs(m):
+    # prefix queries also see the first output
+    orig = m.bidir_prefix_visible_positions
+    m.bidir_prefix_visible_positions = lambda p, L_m, n: (
+        np.arange(1, L_m + 2) if p <= L_m else orig(p, L_m, n))
+
+
 MUTANTS = [
     _mut_window_short, _mut_window_long, _mut_query_index, _mut_prefix_bidirectional,
     _mut_no_scale, _mut_swap_kv, _mut_sign, _mut_softmax_axis, _mut_ring_slot,
     _mut_queue_evicts_reference, _mut_occupancy, _mut_decode_window,
+    _mut_swa_keeps_first_token, _mut_bidir_stays_causal, _mut_bidir_sees_outputs,
 ]
 
 
