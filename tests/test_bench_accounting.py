@@ -1,0 +1,35 @@
+"""The work the benchmark divides by, checked against the oracle's explicit
+sets (CPU): the visible (query, key) pairs behind the prefill FLOP count and
+the cache rows behind the decode byte count."""
+
+from __future__ import annotations
+
+import pytest
+
+import bench
+import oracle
+
+
+@pytest.mark.parametrize("L,L_m,n", [
+    (6, 3, 2), (9, 0, 2), (40, 13, 5), (33, 33, 4), (50, 10, 100), (64, 1, 1), (17, 0, 40),
+])
+def test_visible_pairs_counts_the_packed_mask(L, L_m, n):
+    assert bench.visible_pairs(L, L_m, n) == int(oracle.packed_mask(L, L_m, n).sum())
+
+
+def test_visible_pairs_at_the_32k_config():
+    # the closed form at the full config agrees with a row-by-row count of
+    # the visible sets (without building the 32K x 32K mask)
+    L, L_m, n = 32768, 12832, 128
+    rows = sum(min(p, L_m) if p <= L_m else L_m + min(n, p - L_m) for p in range(1, L + 1))
+    assert bench.visible_pairs(L, L_m, n) == rows == 340_698_960
+
+
+def test_decode_bytes_per_launch_match_the_occupancy_law():
+    # K and V rows of Eq.(6) at T >= n, plus q, o, k_new, v_new
+    w = dict(bench.WORKLOADS["single_doc"])
+    lens = bench.ref_lens_for(w)
+    rows = sum(oracle.occupancy_rswa(w["n"] + 1, L, w["n"]) for L in lens)
+    s = 2  # bf16
+    want = w["H"] * (2 * rows * w["d"] * s) + w["B"] * w["H"] * 4 * w["d"] * s
+    assert bench.bytes_per_launch(w, lens) == want == 13_936_640
