@@ -233,6 +233,28 @@ rswa_status rswa_decode_noalloc(const void* k_cache, const void* v_cache, int S_
                                 void* stream);
 
 /* ------------------------------------------------------------------------
+ * Introspection (host only; needs no device).
+ *
+ * The decode launch plan a handle with these sizes uses, for inspection and
+ * tests.  ref_lens: HOST int32[batch] (each >= 1); window_rows: output rows
+ * the plan covers (n in RSWA mode); S_cap: rows per cache slab; num_sms and
+ * max_clusters: the device's SM count and the resident 8-CTA clusters it
+ * allows (0: never the cluster plan).
+ * Outputs (HOST): items_out int32[items_cap][8], each item
+ *   {bh, row0, rows, part, part_first, nparts, last, 0}: CTA c runs items
+ *   [cta_begin_out[c], cta_begin_out[c+1]) over rows [row0, row0 + rows) of
+ *   slab bh = b*H + h; its partial is number `part` of the slab's `nparts`
+ *   partials starting at `part_first`; `last` marks the slab's last item.
+ * cta_begin_out: int32[cta_cap] (n_ctas + 1 entries).  *cluster_plan is 1
+ * when the slabs are merged inside 8-CTA clusters.  RSWA_ERR_CAPACITY if
+ * items_cap or cta_cap is short.
+ * ---------------------------------------------------------------------- */
+rswa_status rswa_plan_decode(int batch, int H, const int32_t* ref_lens, int window_rows, int S_cap,
+                             int num_sms, int max_clusters, int32_t* items_out, int items_cap,
+                             int32_t* cta_begin_out, int cta_cap, int* n_items, int* n_ctas,
+                             int* cluster_plan);
+
+/* ------------------------------------------------------------------------
  * Misc.
  * ---------------------------------------------------------------------- */
 

@@ -213,6 +213,38 @@ static void make_plan(rswa_ctx* c) {
   c->n_ctas = G;
 }
 
+extern "C" rswa_status rswa_plan_decode(int batch, int H, const int32_t* ref_lens, int window_rows, int S_cap,
+                                        int num_sms, int max_clusters, int32_t* items_out, int items_cap,
+                                        int32_t* cta_begin_out, int cta_cap, int* n_items, int* n_ctas,
+                                        int* cluster_plan) {
+  if (!ref_lens || !items_out || !cta_begin_out || !n_items || !n_ctas || !cluster_plan)
+    return fail(RSWA_ERR_ARG, "rswa_plan_decode: null argument");
+  if (batch < 1 || H < 1 || window_rows < 0 || S_cap < 1 || num_sms < 1 || max_clusters < 0)
+    return fail(RSWA_ERR_ARG, "rswa_plan_decode: invalid sizes");
+  rswa_ctx c{};
+  c.B = batch;
+  c.H = H;
+  c.S_cap = S_cap;
+  c.num_sms = num_sms;
+  c.max_clusters = max_clusters;
+  c.plan_window = window_rows;
+  c.lay = workspace_layout(batch, H, 128);
+  for (int b = 0; b < batch; ++b) {
+    if (ref_lens[b] < 1 || ref_lens[b] > S_cap) return fail(RSWA_ERR_ARG, "rswa_plan_decode: ref_lens[%d]", b);
+    c.Lm.push_back(ref_lens[b]);
+  }
+  make_plan(&c);
+  *n_items = (int)c.items.size();
+  *n_ctas = c.n_ctas;
+  *cluster_plan = c.cluster_plan ? 1 : 0;
+  if ((int)c.items.size() > items_cap || c.n_ctas + 1 > cta_cap)
+    return fail(RSWA_ERR_CAPACITY, "rswa_plan_decode: %zu items, %d CTAs", c.items.size(), c.n_ctas);
+  static_assert(sizeof(DecodeItem) == 8 * sizeof(int32_t), "item layout");
+  memcpy(items_out, c.items.data(), sizeof(DecodeItem) * c.items.size());
+  memcpy(cta_begin_out, c.cta_begin.data(), sizeof(int32_t) * (c.n_ctas + 1));
+  return RSWA_OK;
+}
+
 static rswa_status upload_plan(rswa_ctx* c) {
   if ((int)c->items.size() > c->lay.items_cap)
     return fail(RSWA_ERR_CAPACITY, "decode plan of %zu items exceeds %d", c->items.size(), c->lay.items_cap);
