@@ -125,6 +125,25 @@ rswa_status rswa_init(rswa_handle* out, rswa_mode mode, int L_m_cap, int n, int 
 rswa_status rswa_load_reference(rswa_handle h, const void* K_ref, const void* V_ref,
                                 int ref_stride, const int32_t* ref_lens);
 
+/* Fills the cache from the packed (teacher-forced) layout, so decoding can
+ * continue after a prefill: the result is the cache that
+ * rswa_load_reference followed by T0 appends would leave.  The reference
+ * rows are written once; the ring keeps the newest min(n, T0) outputs, output
+ * t at slot (t-1) mod n (the Eq.(6) cache and its fixed-capacity queue,
+ * 方法展开 §4 and the KV-cache section cited above).
+ *   K, V: device [batch][seq_stride][H][d], the layout rswa_masked_forward
+ *     reads for one sequence ([L][H][d]).  Row p of sequence b is logical
+ *     position p+1: reference rows [0, ref_lens[b]), then output t at row
+ *     ref_lens[b] + t - 1.  Read only; 16-byte aligned.
+ *   ref_lens: HOST array [batch], 1 <= ref_lens[b] <= L_m_cap and
+ *     ref_lens[b] + T0 <= seq_stride.
+ *   T0 >= 0: outputs already produced (the same for every sequence, as the
+ *     step counter is); FULL mode needs T0 <= T_cap.  The next append is
+ *     output T0 + 1.
+ * Stream-ordered; errors are reported before anything is enqueued. */
+rswa_status rswa_load_packed(rswa_handle h, const void* K, const void* V, int seq_stride,
+                             const int32_t* ref_lens, int T0);
+
 /* Appends output T+1 of every sequence: k, v device [batch][H][d].  In RSWA
  * mode the row goes to ring slot (T mod n), overwriting the oldest output
  * once the ring is full (the queue's "position m+1"); in FULL mode to row

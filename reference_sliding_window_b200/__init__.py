@@ -137,6 +137,24 @@ class RSWA:
         self._sync_stream()
         check(_native.lib().rswa_load_reference(self._h, K_ref.data_ptr(), V_ref.data_ptr(), stride, lens))
 
+    def load_packed(self, K: torch.Tensor, V: torch.Tensor, ref_lens: Sequence[int], T0: int) -> None:
+        """Cache as after load_reference + T0 appends, from the packed layout
+        K, V: [B, L, H, d] (or [L, H, d] for one sequence) on the device, where
+        row p of sequence b holds position p+1: the reference rows
+        [0, ref_lens[b]), then output t at row ref_lens[b] + t - 1."""
+        if K.dim() == 3 and self.batch == 1:
+            K, V = K.unsqueeze(0), V.unsqueeze(0)
+        if K.dim() != 4:
+            raise ValueError("K must be [B, L, H, d]")
+        L = K.shape[1]
+        _check_tensor("K", K, (self.batch, L, self.H, self.d), self.dtype, self.device)
+        _check_tensor("V", V, (self.batch, L, self.H, self.d), self.dtype, self.device)
+        if len(ref_lens) != self.batch:
+            raise ValueError("ref_lens must have one entry per sequence")
+        lens = (C.c_int32 * self.batch)(*[int(x) for x in ref_lens])
+        self._sync_stream()
+        check(_native.lib().rswa_load_packed(self._h, K.data_ptr(), V.data_ptr(), L, lens, int(T0)))
+
     def append(self, k: torch.Tensor, v: torch.Tensor) -> None:
         self._vec("k", k)
         self._vec("v", v)

@@ -25,6 +25,7 @@ _PROTOS = {
     "rswa_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
     "rswa_init": (_i, [C.POINTER(_p), _i, _i, _i, _i, _i, _i, _i, _i, _p, _p, _p, _sz, _p]),
     "rswa_load_reference": (_i, [_p, _p, _p, _i, C.POINTER(C.c_int32)]),
+    "rswa_load_packed": (_i, [_p, _p, _p, _i, C.POINTER(C.c_int32), _i]),
     "rswa_append": (_i, [_p, _p, _p]),
     "rswa_decode": (_i, [_p, _p, _p, _f]),
     "rswa_append_decode": (_i, [_p, _p, _p, _p, _p, _f]),

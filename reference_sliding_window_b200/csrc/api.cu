@@ -407,6 +407,55 @@ extern "C" rswa_status rswa_load_reference(rswa_handle h, const void* K_ref, con
   return RSWA_OK;
 }
 
+extern "C" rswa_status rswa_load_packed(rswa_handle h, const void* K, const void* V, int seq_stride,
+                                        const int32_t* ref_lens, int T0) {
+  if (rswa_status st = check_handle(h)) return st;
+  if (!K || !V || !ref_lens) return fail(RSWA_ERR_ARG, "rswa_load_packed: null argument");
+  if (!aligned16(K) || !aligned16(V))
+    return fail(RSWA_ERR_ARG, "rswa_load_packed: K/V must be 16-byte aligned");
+  if (seq_stride < 1 || T0 < 0)
+    return fail(RSWA_ERR_ARG, "rswa_load_packed: seq_stride=%d T0=%d", seq_stride, T0);
+  if (h->mode == RSWA_MODE_FULL && T0 > h->T_cap)
+    return fail(RSWA_ERR_CAPACITY, "rswa_load_packed: T0=%d above T_cap=%d", T0, h->T_cap);
+  int max_rows = 0;
+  const int W = h->mode == RSWA_MODE_RSWA ? std::min(h->n, T0) : T0;
+  for (int b = 0; b < h->B; ++b) {
+    const int L = ref_lens[b];
+    if (L < 1 || L > h->L_m_cap || (long long)L + T0 > seq_stride)
+      return fail(RSWA_ERR_CAPACITY,
+                  "rswa_load_packed: ref_lens[%d]=%d outside [1, L_m_cap=%d] or ref_lens + T0=%d above seq_stride=%d",
+                  b, L, h->L_m_cap, T0, seq_stride);
+    max_rows = std::max(max_rows, L + W);
+  }
+  if (rswa_status st = use_device(h)) return st;
+  h->Lm.assign(ref_lens, ref_lens + h->B);
+  h->T_host = T0;
+  h->plan_window = h->mode == RSWA_MODE_RSWA ? h->n : std::min(h->T_cap, std::max(64, (T0 + 63) / 64 * 64));
+  make_plan(h);
+  RSWA_CUDA(cudaMemcpyAsync(h->ws + h->lay.Lm, h->Lm.data(), 4 * (size_t)h->B, cudaMemcpyHostToDevice,
+                            h->stream),
+            "upload reference lengths");
+  if (rswa_status st = upload_plan(h)) return st;
+  LoadPackedParams p;
+  p.kc = h->kc;
+  p.vc = h->vc;
+  p.K = K;
+  p.V = V;
+  p.B = h->B;
+  p.H = h->H;
+  p.S_cap = h->S_cap;
+  p.row_bytes = h->row_bytes;
+  p.seq_stride = seq_stride;
+  p.n = h->n;
+  p.T0 = T0;
+  p.full_mode = h->mode == RSWA_MODE_FULL;
+  p.Lm = ws_i32(h, h->lay.Lm);
+  p.T = ws_i32(h, h->lay.T);
+  RSWA_CUDA(launch_load_packed(p, max_rows, h->stream), "load_packed kernel");
+  h->loaded = true;
+  return RSWA_OK;
+}
+
 // ------------------------------------------------------------------- steps
 
 static rswa_status check_step(rswa_ctx* c, bool appending, const char* who) {

@@ -70,6 +70,47 @@ __global__ void __launch_bounds__(256) load_reference_kernel(const __grid_consta
   __threadfence();
 }
 
+// grid.y = B*H slabs, grid.x covers the occupied rows x vectors of a slab.
+// Fills the cache as T0 appends after a reference load would have, straight
+// from the packed (teacher-forced) layout, where output t of sequence b is
+// packed row Lm[b] + t - 1.  Cache row Lm[b] + s (ring slot s) holds the
+// newest output t <= T0 with (t - 1) mod n == s; the ring keeps outputs
+// T0-W+1 .. T0, W = min(n, T0), so t - 1 = t0 + ((s - t0) mod n) with
+// t0 = T0 - W.  In FULL mode slot s holds output s + 1.
+__global__ void __launch_bounds__(256) load_packed_kernel(const __grid_constant__ LoadPackedParams p) {
+  const int bh = blockIdx.y;
+  const int b = bh / p.H, h = bh % p.H;
+  const int Lm = p.Lm[b];
+  const int W = p.full_mode ? p.T0 : min(p.n, p.T0);
+  const int t0 = p.T0 - W;
+  const int vpr = p.row_bytes / 16;
+  const long long n_vec = (long long)(Lm + W) * vpr;
+  const size_t src_row_pitch = (size_t)p.H * p.row_bytes;
+  const uint8_t* ks = static_cast<const uint8_t*>(p.K) + (size_t)b * p.seq_stride * src_row_pitch +
+                      (size_t)h * p.row_bytes;
+  const uint8_t* vs = static_cast<const uint8_t*>(p.V) + (size_t)b * p.seq_stride * src_row_pitch +
+                      (size_t)h * p.row_bytes;
+  uint8_t* kd = static_cast<uint8_t*>(p.kc) + (size_t)bh * p.S_cap * p.row_bytes;
+  uint8_t* vd = static_cast<uint8_t*>(p.vc) + (size_t)bh * p.S_cap * p.row_bytes;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n_vec;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int r = (int)(i / vpr), c = (int)(i % vpr);
+    int src = r;
+    if (r >= Lm && !p.full_mode) {
+      const int s = r - Lm;
+      src = Lm + t0 + ((s - t0 % p.n) + p.n) % p.n;
+    }
+    const size_t so = (size_t)src * src_row_pitch + (size_t)c * 16;
+    const size_t dof = (size_t)r * p.row_bytes + (size_t)c * 16;
+    *reinterpret_cast<uint4*>(kd + dof) = *reinterpret_cast<const uint4*>(ks + so);
+    *reinterpret_cast<uint4*>(vd + dof) = *reinterpret_cast<const uint4*>(vs + so);
+  }
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *p.T = p.T0;
+  // Same contract as load_reference_kernel: decode kernels may copy
+  // reference rows before their dependency wait.
+  __threadfence();
+}
+
 cudaError_t launch_append(const AppendParams& p, cudaStream_t stream) {
   append_kernel<<<1, 256, 0, stream>>>(p);
   return cudaGetLastError();
@@ -82,6 +123,16 @@ cudaError_t launch_load_reference(const LoadRefParams& p, int max_len, cudaStrea
   if (gx < 1) gx = 1;
   dim3 grid((unsigned)gx, (unsigned)(p.B * p.H));
   load_reference_kernel<<<grid, 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_load_packed(const LoadPackedParams& p, int max_rows, cudaStream_t stream) {
+  const long long vecs = (long long)max_rows * (p.row_bytes / 16);
+  long long gx = (vecs + 255) / 256;
+  if (gx > 1024) gx = 1024;
+  if (gx < 1) gx = 1;
+  dim3 grid((unsigned)gx, (unsigned)(p.B * p.H));
+  load_packed_kernel<<<grid, 256, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

@@ -91,6 +91,7 @@ def test_init_rejects_bad_arguments_before_device(lib):
 
 def test_null_handle_is_an_argument_error(lib):
     assert lib.rswa_append(None, None, None) == _native.ERR_ARG
+    assert lib.rswa_load_packed(None, None, None, 1, None, 0) == _native.ERR_ARG
     assert lib.rswa_decode(None, None, None, 0.0) == _native.ERR_ARG
     assert lib.rswa_append_decode(None, None, None, None, None, 0.0) == _native.ERR_ARG
     assert lib.rswa_reset(None) == _native.ERR_ARG
