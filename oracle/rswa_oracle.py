@@ -45,6 +45,12 @@ R6  L_m = 0 in the packed form leaves no reference segment: every query p
 R7  Bidirectional prefix (an option; the pages are silent and R2 is the
     default): every prefix query p <= L_m sees all of P = 1..L_m; outputs
     are unchanged.
+R8  Several documents in one pack ([UOW-1] 实验与证据 §1 训练设置: samples
+    are packed to 32K tokens).  The pages do not say how packed documents
+    see each other; we take the plain reading: document i occupies packed
+    rows cu_seqlens[i] .. cu_seqlens[i+1]-1 with its own reference length
+    ref_lens[i], its queries see only its own keys, and inside it the
+    single-sequence mask applies at local positions.
 """
 
 from __future__ import annotations
@@ -64,6 +70,10 @@ __all__ = [
     "attend",
     "masked_forward",
     "masked_forward_rows",
+    "varlen_visible_positions",
+    "varlen_mask",
+    "masked_forward_varlen",
+    "masked_forward_varlen_rows",
     "decode_visible_positions",
     "decode_step",
     "occupancy_rswa",
@@ -280,6 +290,87 @@ def masked_forward_rows(Q: np.ndarray, K: np.ndarray, V: np.ndarray, L_m: int, n
     out = np.empty((len(rows), H, d), dtype=np.float64)
     for i, r in enumerate(rows):
         vis = (bidir_prefix_visible_positions if bidir_prefix else packed_visible_positions)(int(r) + 1, L_m, n) - 1
+        for h in range(H):
+            out[i, h] = attend(Q[r, h], K[vis, h], V[vis, h], sc)
+    return out
+
+
+# --------------------------------------------------------------------------
+# Several documents per pack (reading R8).
+# --------------------------------------------------------------------------
+
+def _check_docs(cu_seqlens: Sequence[int], ref_lens: Sequence[int], n: int) -> List[int]:
+    cu = [int(x) for x in cu_seqlens]
+    if len(cu) < 2 or cu[0] != 0 or len(ref_lens) != len(cu) - 1:
+        raise ValueError("cu_seqlens must start at 0 and have one more entry than ref_lens")
+    for i in range(len(cu) - 1):
+        if cu[i + 1] <= cu[i]:
+            raise ValueError("every document needs at least one row")
+        if not 0 <= int(ref_lens[i]) <= cu[i + 1] - cu[i]:
+            raise ValueError("ref_lens[i] must lie in [0, document length]")
+    if n < 1:
+        raise ValueError("n must be >= 1")
+    return cu
+
+
+def varlen_visible_positions(g: int, cu_seqlens: Sequence[int], ref_lens: Sequence[int], n: int,
+                             bidir_prefix: bool = False) -> np.ndarray:
+    """Keys (1-based pack positions) visible to the query at pack position g:
+    find g's document, apply the single-sequence visible set at the local
+    position, shift back to pack positions (reading R8)."""
+    cu = _check_docs(cu_seqlens, ref_lens, n)
+    if not 1 <= g <= cu[-1]:
+        raise ValueError("g outside the pack")
+    i = next(k for k in range(len(cu) - 1) if cu[k] < g <= cu[k + 1])
+    vis = bidir_prefix_visible_positions if bidir_prefix else packed_visible_positions
+    return vis(g - cu[i], int(ref_lens[i]), n) + cu[i]
+
+
+def varlen_mask(cu_seqlens: Sequence[int], ref_lens: Sequence[int], n: int,
+                bidir_prefix: bool = False) -> np.ndarray:
+    """Explicit [L, L] mask of a pack, L = cu_seqlens[-1]."""
+    L = int(cu_seqlens[-1])
+    M = np.zeros((L, L), dtype=bool)
+    for g in range(1, L + 1):
+        M[g - 1, varlen_visible_positions(g, cu_seqlens, ref_lens, n, bidir_prefix) - 1] = True
+    return M
+
+
+def masked_forward_varlen(Q: np.ndarray, K: np.ndarray, V: np.ndarray, cu_seqlens: Sequence[int],
+                          ref_lens: Sequence[int], n: int, scale=None,
+                          bidir_prefix: bool = False) -> np.ndarray:
+    """Teacher-forced form over a pack of documents: softmax(Q K^T * scale + M) V
+    per head with M = ``varlen_mask`` over the whole pack.
+    Q, K, V: [L, H, d], L = cu_seqlens[-1]  ->  O: [L, H, d] float64."""
+    Q = np.asarray(Q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    L, H, d = Q.shape
+    if L != int(cu_seqlens[-1]):
+        raise ValueError("Q rows must equal cu_seqlens[-1]")
+    sc = _default_scale(d, scale)
+    M = varlen_mask(cu_seqlens, ref_lens, n, bidir_prefix)
+    O = np.empty((L, H, d), dtype=np.float64)
+    for h in range(H):
+        S = (Q[:, h, :] @ K[:, h, :].T) * sc
+        S = np.where(M, S, -np.inf)
+        S = S - S.max(axis=1, keepdims=True)
+        W = np.exp(S)
+        W = W / W.sum(axis=1, keepdims=True)
+        O[:, h, :] = W @ V[:, h, :]
+    return O
+
+
+def masked_forward_varlen_rows(Q: np.ndarray, K: np.ndarray, V: np.ndarray, cu_seqlens: Sequence[int],
+                               ref_lens: Sequence[int], n: int, rows: Sequence[int], scale=None,
+                               bidir_prefix: bool = False) -> np.ndarray:
+    """``masked_forward_varlen`` for the selected 0-based pack rows only.
+    -> [len(rows), H, d]."""
+    L, H, d = Q.shape
+    sc = _default_scale(d, scale)
+    out = np.empty((len(rows), H, d), dtype=np.float64)
+    for i, r in enumerate(rows):
+        vis = varlen_visible_positions(int(r) + 1, cu_seqlens, ref_lens, n, bidir_prefix) - 1
         for h in range(H):
             out[i, h] = attend(Q[r, h], K[vis, h], V[vis, h], sc)
     return out

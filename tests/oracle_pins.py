@@ -341,4 +341,60 @@ def pin_full_mode(o):
     assert not np.allclose(a, b)
 
 
+# ------------------------------------------------- several documents per pack
+
+def pin_varlen_mask_small(o):
+    want = np.array(_rows("varlen_mask_docs_5_4_3_n2.txt"), dtype=bool)
+    got = o.varlen_mask([0, 5, 9, 12], [2, 1, 0], 2)
+    assert got.shape == want.shape and (got == want).all(), got.astype(int)
+
+
+def pin_varlen_predicate(o):
+    # Brute-force predicate, written independently of the set construction:
+    # same document, and j <= p and (j <= L_m or j > p - n) at local positions.
+    rng = np.random.default_rng(61)
+    for _ in range(12):
+        lens = rng.integers(1, 9, rng.integers(1, 5)).tolist()
+        refs = [int(rng.integers(0, x + 1)) for x in lens]
+        n = int(rng.integers(1, 6))
+        cu = np.concatenate([[0], np.cumsum(lens)]).tolist()
+        doc = np.repeat(np.arange(len(lens)), lens)
+        M = o.varlen_mask(cu, refs, n)
+        for g in range(cu[-1]):
+            for k in range(cu[-1]):
+                i = doc[g]
+                p, j, L_m = g - cu[i] + 1, k - cu[i] + 1, refs[i]
+                want = doc[k] == i and j <= p and (j <= L_m or j > p - n)
+                assert bool(M[g, k]) == want, (cu, refs, n, g, k)
+
+
+def pin_varlen_single_document(o):
+    # One document is the single-sequence packed form.
+    for L, L_m, n in ((6, 3, 2), (9, 0, 3), (7, 7, 1), (11, 4, 20)):
+        for bidir in (False, True):
+            assert (o.varlen_mask([0, L], [L_m], n, bidir) == o.packed_mask(L, L_m, n, bidir)).all()
+
+
+def pin_varlen_documents_independent(o):
+    # The pack's output is each document's own output, and a document's
+    # output does not move when another document's K/V change.
+    lens, refs, n, H, d = [7, 3, 9], [3, 0, 9], 2, 2, 4
+    cu = np.concatenate([[0], np.cumsum(lens)]).tolist()
+    Q, K, V = _rand((cu[-1], H, d), 62), _rand((cu[-1], H, d), 63), _rand((cu[-1], H, d), 64)
+    got = o.masked_forward_varlen(Q, K, V, cu, refs, n)
+    for i in range(len(lens)):
+        a, b = cu[i], cu[i + 1]
+        want = o.masked_forward(Q[a:b], K[a:b], V[a:b], refs[i], n)
+        assert np.allclose(got[a:b], want, rtol=1e-13, atol=1e-13), i
+    K2, V2 = K.copy(), V.copy()
+    K2[cu[1]:cu[2]] += 5.0
+    V2[cu[1]:cu[2]] -= 3.0
+    got2 = o.masked_forward_varlen(Q, K2, V2, cu, refs, n)
+    keep = np.r_[0:cu[1], cu[2]:cu[3]]
+    assert np.array_equal(got2[keep], got[keep])
+    rows = [0, cu[1] - 1, cu[1], cu[2], cu[3] - 1]
+    sub = o.masked_forward_varlen_rows(Q, K, V, cu, refs, n, rows)
+    assert np.allclose(sub, got[rows], rtol=1e-13, atol=1e-13)
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -143,11 +143,39 @@ def _mut_bidir_sees_outputs(m):
         np.arange(1, L_m + 2) if p <= L_m else orig(p, L_m, n))
 
 
+def _mut_varlen_global_positions(m):
+    # forgets to shift a document's local positions back to pack positions
+    def varlen_visible_positions(g, cu_seqlens, ref_lens, n, bidir_prefix=False):
+        cu = [int(x) for x in cu_seqlens]
+        i = next(k for k in range(len(cu) - 1) if cu[k] < g <= cu[k + 1])
+        return m.packed_visible_positions(g, int(ref_lens[i]), n)
+    m.varlen_visible_positions = varlen_visible_positions
+
+
+def _mut_varlen_crosses_documents(m):
+    # the whole pack treated as one sequence with the first document's L_m
+    m.varlen_mask = lambda cu, refs, n, bidir_prefix=False: m.packed_mask(int(cu[-1]), int(refs[0]), n,
+                                                                        bidir_prefix)
+
+
+def _mut_varlen_wrong_document(m):
+    # a query on a document's first row is taken as the last row of the previous one
+    orig = m.varlen_visible_positions
+
+    def varlen_visible_positions(g, cu_seqlens, ref_lens, n, bidir_prefix=False):
+        cu = [int(x) for x in cu_seqlens]
+        if g - 1 in cu[1:-1]:
+            return orig(g - 1, cu_seqlens, ref_lens, n, bidir_prefix)
+        return orig(g, cu_seqlens, ref_lens, n, bidir_prefix)
+    m.varlen_visible_positions = varlen_visible_positions
+
+
 MUTANTS = [
     _mut_window_short, _mut_window_long, _mut_query_index, _mut_prefix_bidirectional,
     _mut_no_scale, _mut_swap_kv, _mut_sign, _mut_softmax_axis, _mut_ring_slot,
     _mut_queue_evicts_reference, _mut_occupancy, _mut_decode_window,
     _mut_swa_keeps_first_token, _mut_bidir_stays_causal, _mut_bidir_sees_outputs,
+    _mut_varlen_global_positions, _mut_varlen_crosses_documents, _mut_varlen_wrong_document,
 ]
 
 
@@ -165,6 +193,9 @@ def test_pins_catch_planted_mistake(mutate):
 
 
 def test_oracle_rejects_bad_arguments():
+    for cu, refs in (([1, 4], [1]), ([0, 4, 4], [1, 0]), ([0, 4], [5]), ([0, 4], [1, 1]), ([0, 3], [-1])):
+        with pytest.raises(ValueError):
+            oracle.varlen_mask(cu, refs, 2)
     with pytest.raises(ValueError):
         oracle.window_positions(0, 3, 2)
     with pytest.raises(ValueError):
