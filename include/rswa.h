@@ -221,6 +221,25 @@ rswa_status rswa_masked_forward_ex(const void* Q, const void* K, const void* V, 
                                    int L, int L_m, int n, int H, int d, rswa_dtype dtype,
                                    float scale, int flags, void* stream);
 
+/* The teacher-forced form over a pack of several documents.  The pages pack
+ * training samples to 32K tokens ("Unlimited OCR Works", 实验与证据 §1) and do
+ * not say how packed documents see each other; here each document is its own
+ * sequence: its queries see only its own keys, under the mask above with its
+ * own L_m, at positions local to the document.
+ *   Q, K, V, O: device [L][H][d], L = cu_seqlens[n_docs]; document i holds
+ *     rows [cu_seqlens[i], cu_seqlens[i+1]).
+ *   cu_seqlens: HOST int32[n_docs + 1], cu_seqlens[0] = 0, strictly
+ *     increasing (every document has at least one row).
+ *   ref_lens: HOST int32[n_docs], 0 <= ref_lens[i] <= length of document i.
+ *   n_docs >= 1; n, H, d, dtype, scale, flags as in rswa_masked_forward_ex.
+ * Every argument is checked before anything is enqueued.  The documents are
+ * launched one after another on `stream`, each exactly as
+ * rswa_masked_forward_ex on its rows. */
+rswa_status rswa_masked_forward_varlen(const void* Q, const void* K, const void* V, void* O,
+                                       const int32_t* cu_seqlens, const int32_t* ref_lens, int n_docs,
+                                       int n, int H, int d, rswa_dtype dtype, float scale, int flags,
+                                       void* stream);
+
 /* ------------------------------------------------------------------------
  * Decode without allocation.  The pages have no counterpart to this call;
  * it exists for callers that cannot allocate device memory: a plugin inside

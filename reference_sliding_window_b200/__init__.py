@@ -23,7 +23,7 @@ import torch
 from . import _native
 from ._native import MODE_FULL, MODE_RSWA, RSWAError, check
 
-__all__ = ["RSWA", "masked_forward", "RSWAError", "MODE_RSWA", "MODE_FULL", "library_version"]
+__all__ = ["RSWA", "masked_forward", "masked_forward_varlen", "RSWAError", "MODE_RSWA", "MODE_FULL", "library_version"]
 
 _DT = {torch.float32: _native.F32, torch.bfloat16: _native.BF16}
 
@@ -232,4 +232,33 @@ def masked_forward(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, L_m: int, 
                                                    L, int(L_m), int(n), H, d, _DT[Q.dtype], float(scale),
                                                    _native.FLAG_BIDIR_PREFIX if bidir_prefix else 0,
                                                    _stream_ptr(Q.device)))
+    return O
+
+
+def masked_forward_varlen(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, cu_seqlens: Sequence[int],
+                          ref_lens: Sequence[int], n: int, scale: float = 0.0,
+                          out: Optional[torch.Tensor] = None, bidir_prefix: bool = False) -> torch.Tensor:
+    """Teacher-forced R-SWA attention over a pack of documents.  Q, K, V, out:
+    [L, H, d] on a B200, L = cu_seqlens[-1]; document i holds rows
+    cu_seqlens[i] .. cu_seqlens[i+1]-1 with ref_lens[i] reference rows and
+    sees only its own keys."""
+    if Q.dim() != 3:
+        raise ValueError("Q must be [L, H, d]")
+    L, H, d = Q.shape
+    if Q.dtype not in _DT:
+        raise ValueError(f"dtype {Q.dtype} not supported")
+    n_docs = len(ref_lens)
+    if len(cu_seqlens) != n_docs + 1 or int(cu_seqlens[-1]) != L:
+        raise ValueError("cu_seqlens must have len(ref_lens) + 1 entries ending at L")
+    for name, t in (("Q", Q), ("K", K), ("V", V)):
+        _check_tensor(name, t, (L, H, d), Q.dtype, Q.device)
+    O = torch.empty_like(Q) if out is None else out
+    _check_tensor("out", O, (L, H, d), Q.dtype, Q.device)
+    cu = (C.c_int32 * (n_docs + 1))(*[int(x) for x in cu_seqlens])
+    refs = (C.c_int32 * n_docs)(*[int(x) for x in ref_lens])
+    with torch.cuda.device(Q.device):
+        check(_native.lib().rswa_masked_forward_varlen(
+            Q.data_ptr(), K.data_ptr(), V.data_ptr(), O.data_ptr(), cu, refs, n_docs, int(n), H, d,
+            _DT[Q.dtype], float(scale), _native.FLAG_BIDIR_PREFIX if bidir_prefix else 0,
+            _stream_ptr(Q.device)))
     return O

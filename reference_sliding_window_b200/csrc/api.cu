@@ -709,6 +709,45 @@ extern "C" rswa_status rswa_masked_forward_ex(const void* Q, const void* K, cons
   return RSWA_OK;
 }
 
+extern "C" rswa_status rswa_masked_forward_varlen(const void* Q, const void* K, const void* V, void* O,
+                                                  const int32_t* cu_seqlens, const int32_t* ref_lens,
+                                                  int n_docs, int n, int H, int d, rswa_dtype dtype,
+                                                  float scale, int flags, void* stream) {
+  if (!Q || !K || !V || !O || !cu_seqlens || !ref_lens)
+    return fail(RSWA_ERR_ARG, "rswa_masked_forward_varlen: null argument");
+  if (n_docs < 1) return fail(RSWA_ERR_ARG, "rswa_masked_forward_varlen: n_docs=%d", n_docs);
+  if (flags & ~(int)RSWA_FLAG_BIDIR_PREFIX)
+    return fail(RSWA_ERR_ARG, "rswa_masked_forward_varlen: unknown flags %d", flags);
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
+    return fail(RSWA_ERR_ARG, "rswa_masked_forward_varlen: tensors must be 16-byte aligned");
+  if (!dtype_ok(dtype)) return fail(RSWA_ERR_UNSUPPORTED, "rswa_masked_forward_varlen: unknown dtype");
+  if (d != 64 && d != 128) return fail(RSWA_ERR_UNSUPPORTED, "rswa_masked_forward_varlen: head dim %d", d);
+  if (H < 1 || n < 1) return fail(RSWA_ERR_ARG, "rswa_masked_forward_varlen: H=%d n=%d", H, n);
+  if (!(scale == scale) || isinf(scale)) return fail(RSWA_ERR_ARG, "rswa_masked_forward_varlen: scale not finite");
+  if (cu_seqlens[0] != 0) return fail(RSWA_ERR_ARG, "rswa_masked_forward_varlen: cu_seqlens[0] must be 0");
+  for (int i = 0; i < n_docs; ++i) {
+    const long long len = (long long)cu_seqlens[i + 1] - cu_seqlens[i];
+    if (len < 1)
+      return fail(RSWA_ERR_ARG, "rswa_masked_forward_varlen: document %d has %lld rows", i, len);
+    if (ref_lens[i] < 0 || ref_lens[i] > len)
+      return fail(RSWA_ERR_ARG, "rswa_masked_forward_varlen: ref_lens[%d]=%d outside [0, %lld]", i,
+                  ref_lens[i], len);
+  }
+  if ((long long)cu_seqlens[n_docs] * H * d >= (1ll << 31))
+    return fail(RSWA_ERR_ARG, "rswa_masked_forward_varlen: tensor too large");
+  // Each document is a contiguous [len][H][d] slice of the pack.
+  const size_t row_bytes = (size_t)H * d * elem_size(dtype);
+  for (int i = 0; i < n_docs; ++i) {
+    const size_t off = (size_t)cu_seqlens[i] * row_bytes;
+    rswa_status st = rswa_masked_forward_ex(static_cast<const uint8_t*>(Q) + off, static_cast<const uint8_t*>(K) + off,
+                                            static_cast<const uint8_t*>(V) + off, static_cast<uint8_t*>(O) + off,
+                                            cu_seqlens[i + 1] - cu_seqlens[i], ref_lens[i], n, H, d, dtype,
+                                            scale, flags, stream);
+    if (st != RSWA_OK) return st;
+  }
+  return RSWA_OK;
+}
+
 // -------------------------------------------------------------------- misc
 
 extern "C" const char* rswa_last_error(void) { return g_last_error.c_str(); }

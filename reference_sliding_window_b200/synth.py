@@ -56,6 +56,31 @@ def reference_length(pages: int, prompt_tokens: int) -> int:
     return VISION_TOKENS_PER_PAGE * pages + prompt_tokens
 
 
+# Output (text) tokens per page: the pages do not give one.  400 is the ratio
+# of the 32K teacher-forced workload (19936 outputs after a 50-page
+# reference); each document draws its own from 400 x U[0.5, 1.5].
+OUTPUT_TOKENS_PER_PAGE = 400
+
+
+def pack_documents(total: int, seed: int, prompt_tokens: int = 32,
+                   multi_page_share: float = 0.1) -> tuple:
+    """Documents packed back to back into one sequence of ``total`` rows, as
+    the training data is packed to 32K tokens: single-page documents and
+    multi-page ones (2-50 pages) in a 9:1 mix (实验与证据 §1).  Each document is
+    its reference segment (256 per page + prompt) followed by its outputs; the
+    last one is cut where the pack ends.  -> (cu_seqlens, ref_lens)."""
+    rng = np.random.default_rng(seed)
+    cu, refs = [0], []
+    while cu[-1] < total:
+        pages = int(rng.integers(2, 51)) if rng.random() < multi_page_share else 1
+        outs = int(round(OUTPUT_TOKENS_PER_PAGE * pages * rng.uniform(0.5, 1.5)))
+        room = total - cu[-1]
+        L_m = min(reference_length(pages, prompt_tokens), room)
+        cu.append(cu[-1] + min(L_m + outs, room))
+        refs.append(L_m)
+    return cu, refs
+
+
 @dataclass
 class DecodeCase:
     """Inputs of a decode run.

@@ -123,6 +123,35 @@ def test_masked_forward_ex_rejects_unknown_flags(lib):
     assert mfx(None, p, p, p, 8, 2, 2, 1, 64, _native.F32, 0.0, _native.FLAG_BIDIR_PREFIX, None) == _native.ERR_ARG
 
 
+def test_masked_forward_varlen_rejects_bad_arguments_before_device(lib):
+    # Every case fails the host checks, so nothing is launched.
+    buf = C.create_string_buffer(256)
+    p = (C.cast(buf, C.c_void_p).value + 15) // 16 * 16
+    mv = lib.rswa_masked_forward_varlen
+
+    def call(cu, refs, n_docs=None, n=2, H=1, d=64, dtype=_native.F32, scale=0.0, flags=0, Q=p, O=p):
+        cu_a = (C.c_int32 * len(cu))(*cu)
+        refs_a = (C.c_int32 * max(len(refs), 1))(*refs)
+        nd = len(refs) if n_docs is None else n_docs
+        return mv(Q, p, p, O, cu_a, refs_a, nd, n, H, d, dtype, scale, flags, None)
+
+    assert call([0, 4], [1], Q=None) == _native.ERR_ARG
+    assert call([0, 4], [1], O=p + 4) == _native.ERR_ARG
+    assert call([0], [], n_docs=0) == _native.ERR_ARG
+    assert call([0, 4], [1], flags=2) == _native.ERR_ARG
+    assert call([1, 4], [1]) == _native.ERR_ARG          # must start at 0
+    assert call([0, 4, 4], [1, 0]) == _native.ERR_ARG    # empty document
+    assert call([0, 4, 3], [1, 0]) == _native.ERR_ARG    # decreasing
+    assert call([0, 4], [5]) == _native.ERR_ARG          # more reference rows than rows
+    assert call([0, 4, 6], [1, -1]) == _native.ERR_ARG
+    assert call([0, 4], [1], n=0) == _native.ERR_ARG
+    assert call([0, 4], [1], H=0) == _native.ERR_ARG
+    assert call([0, 4], [1], d=80) == _native.ERR_UNSUPPORTED
+    assert call([0, 4], [1], dtype=3) == _native.ERR_UNSUPPORTED
+    assert call([0, 4], [1], scale=float("inf")) == _native.ERR_ARG
+    assert call([0, 1 << 30], [0], H=4) == _native.ERR_ARG  # 2^31 elements or more
+
+
 def test_product_path_has_no_oracle_dependency():
     # The package must never import the oracle (or any CPU fallback).
     pkg = os.path.join(ROOT, "reference_sliding_window_b200")
