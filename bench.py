@@ -67,6 +67,12 @@ def visible_pairs(L, L_m, n):
     return L_m * (L_m + 1) // 2 + T_out * L_m + sum(min(n, t) for t in range(1, T_out + 1))
 
 
+def visible_keys(r, L_m, n):
+    """Keys visible to 0-based query row r of the packed mask: causal in the
+    prefix, else the L_m reference keys plus the window of n."""
+    return r + 1 if r < L_m else L_m + min(n, r - L_m + 1)
+
+
 def log(*a):
     print(*a, file=sys.stderr, flush=True)
 
@@ -473,6 +479,35 @@ def oracle_sample(w, lens, budget_s: float, seed: int = 0):
     return B * steps / el, threads, f"{steps} decode steps x {B} sequences x {H} heads (T={T}), fp64 numpy"
 
 
+def oracle_prefill_sample(w, budget_s: float, seed: int = 0, n_random: int = 256):
+    """Times the fp64 CPU oracle on sampled query rows of the teacher-forced
+    workload: the rows at the segment edges, then random rows, one at a time
+    until the budget is spent.  Returns (algorithmic TFLOP/s over the visible
+    pairs of the rows done, threads, description)."""
+    import numpy as np
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = 1
+    rng = np.random.default_rng(seed)
+    L, L_m, n, H, d = w["L"], w["L_m"], w["n"], w["H"], w["d"]
+    Q, K, V = (rng.standard_normal((L, H, d), dtype=np.float32) for _ in range(3))
+    edges = [0, L_m - 1, L_m, L_m + n - 1, L_m + n, L - 1]
+    rows = [r for r in edges if 0 <= r < L] + rng.integers(0, L, n_random).tolist()
+    done, pairs, t0 = 0, 0, time.perf_counter()
+    for r in rows:
+        oracle.masked_forward_rows(Q, K, V, L_m, n, [r])
+        pairs += visible_keys(r, L_m, n)
+        done += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s and done >= 2:
+            break
+    return (4.0 * d * pairs * H / el / 1e12, threads,
+            f"{done} query rows (segment edges, then random) x {H} heads of the {L}-row pack, fp64 numpy")
+
+
 # -------------------------------------------------------------------- main
 
 def main():
@@ -569,18 +604,36 @@ def main():
 
 def main_prefill(args):
     """--workload prefill: the teacher-forced form on its own JSON line."""
-    import torch
     world, rank, local = dist_env()
     if rank != 0:
         return 0
+    metric = "R-SWA masked prefill TFLOP/s (algorithmic, visible pairs only)"
+    if args.impl == "reference":
+        v, threads, sample = oracle_prefill_sample(PREFILL, args.cpu_budget)
+        line = {"metric": metric, "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+                "warmup": args.warmup,
+                # one whole call's algorithmic FLOPs at the sampled rate
+                "ms_per_step": 1e3 * 4.0 * PREFILL["d"] * PREFILL["H"] *
+                visible_pairs(PREFILL["L"], PREFILL["L_m"], PREFILL["n"]) / (v * 1e12),
+                "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+                "config": {"workload": PREFILL["desc"], "l2": "host CPU"},
+                "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                                 "sample": sample},
+                "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return 0
+    import torch
     torch.cuda.set_device(local)
     r = run_prefill(max(1, args.steps), max(3, args.warmup))
-    line = {"metric": "R-SWA masked prefill TFLOP/s (algorithmic, visible pairs only)", "value": r["tflops"],
+    v, threads, sample = oracle_prefill_sample(PREFILL, args.cpu_budget)
+    line = {"metric": metric, "value": r["tflops"],
             "unit": "TFLOP/s", "n_gpus": 1, "steps": r["iters"], "warmup": max(3, args.warmup),
             "ms_per_step": r["ms_per_call"], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
             "config": {"workload": r["workload"], "l2": "inputs 252 MB, larger than L2"},
-            "roofline": r["roofline"], "gpu_launches": r["iters"]}
+            "roofline": r["roofline"], "gpu_launches": r["iters"],
+            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": sample}}
     print(json.dumps(line), flush=True)
     return 0
 

@@ -33,3 +33,16 @@ def test_decode_bytes_per_launch_match_the_occupancy_law():
     s = 2  # bf16
     want = w["H"] * (2 * rows * w["d"] * s) + w["B"] * w["H"] * 4 * w["d"] * s
     assert bench.bytes_per_launch(w, lens) == want == 13_936_640
+
+
+@pytest.mark.parametrize("L,L_m,n", [(6, 3, 2), (40, 13, 5), (50, 10, 100), (17, 0, 4)])
+def test_visible_keys_per_row_match_the_oracle(L, L_m, n):
+    # the per-row count behind the prefill oracle baseline's FLOPs
+    for r in range(L):
+        assert bench.visible_keys(r, L_m, n) == len(oracle.packed_visible_positions(r + 1, L_m, n)), r
+
+
+def test_prefill_oracle_baseline_runs_on_a_small_pack():
+    w = dict(L=300, L_m=100, n=16, H=2, d=16)
+    v, threads, sample = bench.oracle_prefill_sample(w, budget_s=0.05, n_random=8)
+    assert v > 0 and threads >= 1 and "query rows" in sample
