@@ -158,7 +158,13 @@ rswa_status rswa_decode(rswa_handle h, const void* q, void* o, float scale);
 /* rswa_append followed by rswa_decode in ONE kernel: the new k, v are
  * written in place into their slot (no compaction copy) while the cache is
  * streamed, and the step counter is advanced on the device, so a captured
- * CUDA graph of this call can be replayed step after step. */
+ * CUDA graph of this call can be replayed step after step.  In FULL mode
+ * the launch plan is made on the host and covers outputs up to the first
+ * multiple of 64 at or above the next output; a graph replayed beyond that
+ * finds more rows than its plan, and rswa_check then returns
+ * RSWA_ERR_DEVICE ("plan-short") rather than the step attending to a
+ * subset: re-capture FULL-mode graphs within that range.  RSWA mode has no
+ * such limit (its plan covers the whole ring). */
 rswa_status rswa_append_decode(rswa_handle h, const void* k, const void* v,
                                const void* q, void* o, float scale);
 
