@@ -131,9 +131,9 @@ class RSWA:
         stride = K_ref.shape[2]
         _check_tensor("K_ref", K_ref, (self.batch, self.H, stride, self.d), self.dtype, self.device)
         _check_tensor("V_ref", V_ref, (self.batch, self.H, stride, self.d), self.dtype, self.device)
-        lens = (C.c_int32 * self.batch)(*[int(x) for x in ref_lens])
         if len(ref_lens) != self.batch:
             raise ValueError("ref_lens must have one entry per sequence")
+        lens = (C.c_int32 * self.batch)(*[int(x) for x in ref_lens])
         self._sync_stream()
         check(_native.lib().rswa_load_reference(self._h, K_ref.data_ptr(), V_ref.data_ptr(), stride, lens))
 
