@@ -14,6 +14,7 @@
 #include <string>
 #include <vector>
 
+#include "cache_copy.h"
 #include "internal.h"
 #include "rswa.h"
 

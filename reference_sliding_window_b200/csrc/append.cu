@@ -9,6 +9,7 @@
 // ("position m+1", same page, KV cache 恒定 section); in FULL mode slot = T-1.
 // Rows are moved as 16-byte vectors (row sizes are multiples of 128 bytes).
 
+#include "cache_copy.h"
 #include "common.cuh"
 #include "internal.h"
 
