@@ -53,8 +53,18 @@ def _rank_main(rank: int, port: int, out) -> None:
         finally:
             sys.argv = argv
         dist.barrier()
+        # the prefill workload's reference arm follows the same rule
+        pbuf = io.StringIO()
+        sys.argv = ["bench.py", "--impl", "reference", "--workload", "prefill", "--gpus", str(WORLD),
+                    "--steps", "4", "--warmup", "3", "--cpu-budget", "0.05"]
+        try:
+            with contextlib.redirect_stdout(pbuf):
+                prc = bench.main()
+        finally:
+            sys.argv = argv
+        dist.barrier()
         out.put({"rank": rank, "env": env, "el_max": el_max, "tok_sum": tok_sum, "seeds": seeds,
-                 "rc": rc, "stdout": buf.getvalue()})
+                 "rc": rc, "stdout": buf.getvalue(), "prefill_rc": prc, "prefill_stdout": pbuf.getvalue()})
     finally:
         dist.destroy_process_group()
 
@@ -113,3 +123,13 @@ def test_reference_arm_runs_on_rank0_only(ranks):
 def test_single_process_reduction_is_identity():
     import bench
     assert bench.reduce_max_sum(0.25, 7.0) == (0.25, 7.0)
+
+
+def test_prefill_reference_arm_runs_on_rank0_only(ranks):
+    assert ranks[0]["prefill_rc"] == 0 and ranks[1]["prefill_rc"] == 0
+    assert ranks[1]["prefill_stdout"].strip() == ""
+    lines = [ln for ln in ranks[0]["prefill_stdout"].splitlines() if ln.strip()]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["unit"] == "TFLOP/s" and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["ms_per_step"] > 0
