@@ -80,3 +80,24 @@ def test_varlen_rejects_bad_documents():
         masked_forward_varlen(Q, Q, Q, [0, 8, 16], [9, 1], 2)   # more reference rows than rows
     with pytest.raises(RSWAError, match="ARG"):
         masked_forward_varlen(Q, Q, Q, [0, 8, 8, 16], [1, 0, 1], 2)
+
+
+@pytest.mark.parametrize("L,L_m,n", [(1, 1, 1), (77, 30, 8), (127, 0, 16), (100, 100, 4)])
+def test_tensor_core_kernel_shorter_than_one_tile(L, L_m, n):
+    """bf16, d=128 takes the tensor-core kernel; with L < 128 its only query
+    tile is part padding (the tensor maps zero-fill rows past L)."""
+    Q, K, V = synth.prefill_case(L, 2, 128, "bf16", seed=L + 90)
+    O = masked_forward(Q.cuda(), K.cuda(), V.cuda(), L_m=L_m, n=n)
+    torch.cuda.synchronize()
+    want = oracle.masked_forward(Q.double().numpy(), K.double().numpy(), V.double().numpy(), L_m, n)
+    assert_close(O, want, "bf16", "short sequence, tensor-core kernel")
+
+
+def test_varlen_pack_with_short_documents_on_tensor_cores():
+    cu, refs, n = [0, 5, 133, 200, 201, 500], [5, 60, 0, 1, 288], 16
+    L = cu[-1]
+    Q, K, V = synth.prefill_case(L, 2, 128, "bf16", seed=95)
+    O = masked_forward_varlen(Q.cuda(), K.cuda(), V.cuda(), cu, refs, n)
+    torch.cuda.synchronize()
+    want = oracle.masked_forward_varlen(Q.double().numpy(), K.double().numpy(), V.double().numpy(), cu, refs, n)
+    assert_close(O, want, "bf16", "pack with short documents")
