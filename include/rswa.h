@@ -101,12 +101,13 @@ size_t rswa_workspace_bytes(int L_m_cap, int window_cap, int H, int d, int batch
  *   The caches belong to the handle until rswa_destroy: the caller must not
  *     write them.  Decode kernels copy reference rows before waiting on the
  *     preceding kernel of the stream (programmatic dependent launch); this
- *     is safe because only rswa_load_reference writes those rows and its
- *     kernel makes its writes visible before it retires.
+ *     is safe because only rswa_load_reference and rswa_load_packed write
+ *     those rows and their kernels make their writes visible before they
+ *     retire.
  *   workspace: rswa_workspace_bytes(...) bytes; zeroed by this call
  *     (stream-ordered).
  *   n: window size (RSWA mode, >= 1).  T_cap: max outputs (FULL mode, >= 1).
- *   The other of n / T_cap is ignored.
+ *   The other of n / T_cap is ignored.  batch * H <= 65535.
  *   Decode plan: when every (b, h) slab can have a resident cluster of
  *   8 CTAs, a slab's partial results are merged inside its cluster;
  *   otherwise across CTAs through the workspace.  The environment variable

@@ -297,6 +297,8 @@ extern "C" rswa_status rswa_init(rswa_handle* out, rswa_mode mode, int L_m_cap, 
   if (d != 64 && d != 128) return fail(RSWA_ERR_UNSUPPORTED, "rswa_init: head dim %d (64 or 128)", d);
   if (L_m_cap < 1 || H < 1 || batch < 1)
     return fail(RSWA_ERR_ARG, "rswa_init: L_m_cap=%d H=%d batch=%d must be >= 1", L_m_cap, H, batch);
+  if ((long long)batch * H > 65535)  // one grid row per (b, h) slab in the cache-fill kernels
+    return fail(RSWA_ERR_ARG, "rswa_init: batch*H=%lld above 65535", (long long)batch * H);
   if (mode == RSWA_MODE_RSWA && n < 1) return fail(RSWA_ERR_ARG, "rswa_init: window n=%d must be >= 1", n);
   if (mode == RSWA_MODE_FULL && T_cap < 1)
     return fail(RSWA_ERR_ARG, "rswa_init: T_cap=%d must be >= 1 in FULL mode", T_cap);

@@ -81,6 +81,8 @@ def test_init_rejects_bad_arguments_before_device(lib):
     assert lib.rswa_init(C.byref(h), 1, 10, 4, 0, 2, 64, 1, _native.BF16, p16, p16, p16, 1 << 20, None) == _native.ERR_ARG
     assert "T_cap" in _err(lib)
     assert lib.rswa_init(C.byref(h), 0, 10, 4, 0, 2, 64, 1, _native.BF16, None, p16, p16, 1 << 20, None) == _native.ERR_ARG
+    assert lib.rswa_init(C.byref(h), 0, 10, 4, 0, 256, 64, 257, _native.BF16, p16, p16, p16, 1 << 20, None) == _native.ERR_ARG
+    assert "65535" in _err(lib)
     assert lib.rswa_init(C.byref(h), 0, 10, 4, 0, 2, 64, 1, _native.BF16, p16 + 8, p16, p16, 1 << 20, None) == _native.ERR_ARG
     assert "aligned" in _err(lib)
     assert lib.rswa_init(C.byref(h), 0, 10, 4, 0, 2, 64, 1, _native.BF16, p16, p16, p16, 16, None) == _native.ERR_ARG
