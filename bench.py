@@ -105,6 +105,19 @@ def measured_tensor_peak():
 CURVE_T = (1, 32, 64, 128, 256, 512, 1024, 2048, 4096, 6144)
 
 
+def cache_rows(lens, n, T, full):
+    """Cache rows of one head, summed over the sequences, after T outputs:
+    L_m + min(n, T) each for R-SWA (Eq.(6)), L_m + T with every output kept
+    (Eq.(5))."""
+    return sum((L + T) if full else (L + min(n, T)) for L in lens)
+
+
+def curve_cache_ratio(lens, n, Ts):
+    """R-SWA cache over the full cache at each T (Eq.(7); one sequence gives
+    (L_m + min(n, T)) / (L_m + T))."""
+    return [round(cache_rows(lens, n, T, False) / cache_rows(lens, n, T, True), 6) for T in Ts]
+
+
 def run_curve(w, lens, samples: int = 8):
     """Per-step decode latency against the output length T, for the R-SWA
     cache and for the same kernel over the full cache (every output kept):
@@ -122,7 +135,8 @@ def run_curve(w, lens, samples: int = 8):
     flush = torch.empty(2 * torch.cuda.get_device_properties(dev).L2_cache_size, dtype=torch.uint8, device=dev)
     pool = synth.normal((16, 3, B, H, d), 4000, w["dtype"], "cuda")
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    out = {"T": list(CURVE_T), "samples": samples, "timing": "isolated launches after an L2 flush, median"}
+    out = {"T": list(CURVE_T), "samples": samples, "timing": "isolated launches after an L2 flush, median",
+           "cache_ratio": curve_cache_ratio(lens, n, CURVE_T)}
     for name, mode in (("rswa", MODE_RSWA), ("full", MODE_FULL)):
         a = RSWA(L_m_cap, n, H, d, B, dt, mode=mode, T_cap=T_top, device=dev)
         Kr = synth.normal((B, H, L_m_cap, d), 4100, w["dtype"], "cuda")
@@ -147,7 +161,7 @@ def run_curve(w, lens, samples: int = 8):
                 ts.append(e0.elapsed_time(e1) * 1e3)
                 T += 1
             t_us = statistics.median(ts)
-            rows = sum((L + min(n, Tc)) if mode == MODE_RSWA else (L + Tc) for L in lens)
+            rows = cache_rows(lens, n, Tc, mode == MODE_FULL)
             us.append(round(t_us, 2))
             gbs.append(round(H * (2 * rows * d * s + 4 * B * d * s) / t_us / 1e3, 1))
         a.check()

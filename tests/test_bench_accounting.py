@@ -46,3 +46,18 @@ def test_prefill_oracle_baseline_runs_on_a_small_pack():
     w = dict(L=300, L_m=100, n=16, H=2, d=16)
     v, threads, sample = bench.oracle_prefill_sample(w, budget_s=0.05, n_random=8)
     assert v > 0 and threads >= 1 and "query rows" in sample
+
+
+def test_curve_cache_rows_and_ratio_follow_eq5_to_eq7():
+    w = dict(bench.WORKLOADS["single_doc"])
+    lens = bench.ref_lens_for(w)
+    n = w["n"]
+    for T in bench.CURVE_T:
+        assert bench.cache_rows(lens, n, T, False) == sum(oracle.occupancy_rswa(T, L, n) for L in lens)
+        assert bench.cache_rows(lens, n, T, True) == sum(oracle.occupancy_full(T, L) for L in lens)
+    ratios = bench.curve_cache_ratio(lens, n, bench.CURVE_T)
+    assert len(lens) == 1 and len(ratios) == len(bench.CURVE_T)
+    for T, r in zip(bench.CURVE_T, ratios):
+        assert r == pytest.approx(oracle.cache_ratio(T, lens[0], n), abs=1e-6)
+    # ragged batch: the ratio of summed rows
+    assert bench.curve_cache_ratio([5, 7], 2, [1, 4]) == [1.0, round((7 + 9) / (9 + 11), 6)]
