@@ -142,6 +142,16 @@ def pin_packed_mask_predicate(o):
                 assert bool(M[p - 1, j - 1]) == want, (L_m, n, p, j)
 
 
+def pin_window_of_one_is_reference_plus_self(o):
+    # n = 1: an output query sees P and itself, nothing else (closed form).
+    for L_m in (1, 4, 9):
+        P = list(range(1, L_m + 1))
+        for p in range(L_m + 1, L_m + 7):
+            assert o.packed_visible_positions(p, L_m, 1).tolist() == P + [p], (L_m, p)
+        for T in range(1, 6):
+            assert o.decode_visible_positions(T, L_m, 1).tolist() == P + [L_m + T], (L_m, T)
+
+
 # ----------------------------------------------------------------- numerics
 
 def pin_short_output_is_causal(o):
