@@ -216,6 +216,50 @@ def run_prefill(iters: int, warmup: int):
                                      "tflops": 4.0 * w["d"] * pairs_swa * w["H"] / sec_swa / 1e12}}
 
 
+VARLEN_SEED = 32  # the 32K pack of 10 documents (9 single-page, one of 47 pages)
+
+
+def pack_visible_pairs(cu, refs, n):
+    """Visible (query, key) pairs per head of a pack: each document's own
+    packed mask, nothing across documents."""
+    return sum(visible_pairs(cu[i + 1] - cu[i], refs[i], n) for i in range(len(refs)))
+
+
+def run_varlen(iters: int, warmup: int):
+    """Times rswa_masked_forward_varlen on a 32768-row pack of documents
+    (inputs 252 MB, larger than L2).  Returns a dict for the JSON line."""
+    import torch
+    from reference_sliding_window_b200 import masked_forward_varlen, synth
+    w = PREFILL
+    cu, refs = synth.pack_documents(w["L"], seed=VARLEN_SEED)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    Q, K, V = synth.prefill_case(w["L"], w["H"], w["d"], w["dtype"], seed=22, device="cuda")
+    O = torch.empty_like(Q)
+    for _ in range(max(1, warmup)):
+        masked_forward_varlen(Q, K, V, cu, refs, w["n"], out=O)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(iters):
+        masked_forward_varlen(Q, K, V, cu, refs, w["n"], out=O)
+    e1.record()
+    torch.cuda.synchronize(dev)
+    sec = e0.elapsed_time(e1) / 1e3 / iters
+    pairs = pack_visible_pairs(cu, refs, w["n"])
+    flops = 4.0 * w["d"] * pairs * w["H"]
+    peak, kind = measured_tensor_peak()
+    tf = flops / sec / 1e12
+    return {"workload": f"teacher-forced masked prefill over a pack, bf16: {w['L']} rows holding {len(refs)} "
+                        f"documents (lengths {[cu[i + 1] - cu[i] for i in range(len(refs))]}, L_m {refs}), "
+                        f"10 heads, d=128, n={w['n']}",
+            "ms_per_call": sec * 1e3, "iters": iters, "launches_per_call": len(refs), "tflops": tf,
+            "visible_pairs_per_head": pairs,
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+                         "peak_kind": f"{kind} dense bf16 (burst)", "traffic": None,
+                         "algorithmic_flops_per_launch": flops / len(refs),
+                         "kernel": "rswa::tc::masked_tc_kernel (one launch per document)"}}
+
+
 DECODE_SOURCES = ("decode.cu", "common.cuh", "internal.h")
 PREFILL_SOURCES = ("masked_tc.cu", "common.cuh")  # the kernel takes its parameters from masked_tc.cu
 
@@ -493,9 +537,10 @@ def oracle_sample(w, lens, budget_s: float, seed: int = 0):
     return B * steps / el, threads, f"{steps} decode steps x {B} sequences x {H} heads (T={T}), fp64 numpy"
 
 
-def oracle_prefill_sample(w, budget_s: float, seed: int = 0, n_random: int = 256):
+def oracle_prefill_sample(w, budget_s: float, seed: int = 0, n_random: int = 256, docs=None):
     """Times the fp64 CPU oracle on sampled query rows of the teacher-forced
-    workload: the rows at the segment edges, then random rows, one at a time
+    workload: the rows at the segment edges (of every document, for a pack
+    given as docs = (cu_seqlens, ref_lens)), then random rows, one at a time
     until the budget is spent.  Returns (algorithmic TFLOP/s over the visible
     pairs of the rows done, threads, description)."""
     import numpy as np
@@ -508,18 +553,28 @@ def oracle_prefill_sample(w, budget_s: float, seed: int = 0, n_random: int = 256
     rng = np.random.default_rng(seed)
     L, L_m, n, H, d = w["L"], w["L_m"], w["n"], w["H"], w["d"]
     Q, K, V = (rng.standard_normal((L, H, d), dtype=np.float32) for _ in range(3))
-    edges = [0, L_m - 1, L_m, L_m + n - 1, L_m + n, L - 1]
-    rows = [r for r in edges if 0 <= r < L] + rng.integers(0, L, n_random).tolist()
+    cu, refs = docs if docs is not None else ([0, L], [L_m])
+    doc_of = np.repeat(np.arange(len(refs)), np.diff(cu))
+    edges = []
+    for i, Lm in enumerate(refs):
+        a, b = cu[i], cu[i + 1]
+        edges += [r for r in (a, a + Lm - 1, a + Lm, a + Lm + n - 1, a + Lm + n, b - 1) if a <= r < b]
+    rows = edges + rng.integers(0, L, n_random).tolist()
     done, pairs, t0 = 0, 0, time.perf_counter()
     for r in rows:
-        oracle.masked_forward_rows(Q, K, V, L_m, n, [r])
-        pairs += visible_keys(r, L_m, n)
+        i = int(doc_of[r])
+        if docs is None:
+            oracle.masked_forward_rows(Q, K, V, L_m, n, [r])
+        else:
+            oracle.masked_forward_varlen_rows(Q, K, V, cu, refs, n, [r])
+        pairs += visible_keys(r - cu[i], refs[i], n)
         done += 1
         el = time.perf_counter() - t0
         if el >= budget_s and done >= 2:
             break
+    what = f"{L}-row pack of {len(refs)} documents" if docs is not None else f"{L}-row sequence"
     return (4.0 * d * pairs * H / el / 1e12, threads,
-            f"{done} query rows (segment edges, then random) x {H} heads of the {L}-row pack, fp64 numpy")
+            f"{done} query rows (segment edges, then random) x {H} heads of the {what}, fp64 numpy")
 
 
 # -------------------------------------------------------------------- main
@@ -530,7 +585,7 @@ def main():
     ap.add_argument("--steps", type=int, default=6144)
     ap.add_argument("--warmup", type=int, default=16)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["prefill"], default="single_doc")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["prefill", "varlen"], default="single_doc")
     ap.add_argument("--prefill-iters", type=int, default=10, help="timed masked-prefill calls (0: skip)")
     ap.add_argument("--curve", type=int, default=1, help="1: add per-step latency vs T, R-SWA and full cache")
     ap.add_argument("--layers", type=int, default=0, help="layer caches cycled (0: 2 x L2 rule)")
@@ -541,7 +596,7 @@ def main():
         ap.error("--warmup must be >= 3")
 
     world, rank, local = dist_env()
-    if args.workload == "prefill":
+    if args.workload in ("prefill", "varlen"):
         return main_prefill(args)
     w = WORKLOADS[args.workload]
     lens = ref_lens_for(w)
@@ -617,21 +672,30 @@ def main():
 
 
 def main_prefill(args):
-    """--workload prefill: the teacher-forced form on its own JSON line."""
+    """--workload prefill / varlen: the teacher-forced form, on one sequence
+    or on a pack of documents, on its own JSON line."""
     world, rank, local = dist_env()
     if rank != 0:
         return 0
     metric = "R-SWA masked prefill TFLOP/s (algorithmic, visible pairs only)"
+    docs = None
+    if args.workload == "varlen":
+        from reference_sliding_window_b200 import synth
+        docs = synth.pack_documents(PREFILL["L"], seed=VARLEN_SEED)
+        pairs = pack_visible_pairs(docs[0], docs[1], PREFILL["n"])
+        desc = f"teacher-forced masked prefill over a pack, bf16: {PREFILL['L']} rows, {len(docs[1])} documents"
+    else:
+        pairs = visible_pairs(PREFILL["L"], PREFILL["L_m"], PREFILL["n"])
+        desc = PREFILL["desc"]
     if args.impl == "reference":
-        v, threads, sample = oracle_prefill_sample(PREFILL, args.cpu_budget)
+        v, threads, sample = oracle_prefill_sample(PREFILL, args.cpu_budget, docs=docs)
         line = {"metric": metric, "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
                 "warmup": args.warmup,
                 # one whole call's algorithmic FLOPs at the sampled rate
-                "ms_per_step": 1e3 * 4.0 * PREFILL["d"] * PREFILL["H"] *
-                visible_pairs(PREFILL["L"], PREFILL["L_m"], PREFILL["n"]) / (v * 1e12),
+                "ms_per_step": 1e3 * 4.0 * PREFILL["d"] * PREFILL["H"] * pairs / (v * 1e12),
                 "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-                "config": {"workload": PREFILL["desc"], "l2": "host CPU"},
+                "config": {"workload": desc, "l2": "host CPU"},
                 "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                                  "sample": sample},
                 "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -639,14 +703,19 @@ def main_prefill(args):
         return 0
     import torch
     torch.cuda.set_device(local)
-    r = run_prefill(max(1, args.steps), max(3, args.warmup))
-    v, threads, sample = oracle_prefill_sample(PREFILL, args.cpu_budget)
+    if docs is not None:
+        r = run_varlen(max(1, args.steps), max(3, args.warmup))
+        launches = r["iters"] * r["launches_per_call"]
+    else:
+        r = run_prefill(max(1, args.steps), max(3, args.warmup))
+        launches = r["iters"]
+    v, threads, sample = oracle_prefill_sample(PREFILL, args.cpu_budget, docs=docs)
     line = {"metric": metric, "value": r["tflops"],
             "unit": "TFLOP/s", "n_gpus": 1, "steps": r["iters"], "warmup": max(3, args.warmup),
             "ms_per_step": r["ms_per_call"], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
             "config": {"workload": r["workload"], "l2": "inputs 252 MB, larger than L2"},
-            "roofline": r["roofline"], "gpu_launches": r["iters"],
+            "roofline": r["roofline"], "gpu_launches": launches,
             "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": sample}}
     print(json.dumps(line), flush=True)
     return 0

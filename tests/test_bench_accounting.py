@@ -61,3 +61,16 @@ def test_curve_cache_rows_and_ratio_follow_eq5_to_eq7():
         assert r == pytest.approx(oracle.cache_ratio(T, lens[0], n), abs=1e-6)
     # ragged batch: the ratio of summed rows
     assert bench.curve_cache_ratio([5, 7], 2, [1, 4]) == [1.0, round((7 + 9) / (9 + 11), 6)]
+
+
+@pytest.mark.parametrize("cu,refs,n", [([0, 5, 9, 12], [2, 1, 0], 2), ([0, 30, 31, 80], [10, 1, 49], 4),
+                                       ([0, 17], [17], 3)])
+def test_pack_visible_pairs_count_the_varlen_mask(cu, refs, n):
+    assert bench.pack_visible_pairs(cu, refs, n) == int(oracle.varlen_mask(cu, refs, n).sum())
+
+
+def test_pack_oracle_baseline_runs_on_a_small_pack():
+    w = dict(L=300, L_m=100, n=16, H=2, d=16)
+    v, threads, sample = bench.oracle_prefill_sample(w, budget_s=0.05, n_random=4,
+                                                     docs=([0, 120, 121, 300], [40, 1, 0]))
+    assert v > 0 and "3 documents" in sample
