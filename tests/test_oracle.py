@@ -179,6 +179,8 @@ MUTANTS = [
 ]
 
 
+# a planted mistake can leave a query with no visible key (a row of -inf)
+@pytest.mark.filterwarnings("ignore:invalid value encountered:RuntimeWarning")
 @pytest.mark.parametrize("mutate", MUTANTS, ids=lambda f: f.__name__[5:])
 def test_pins_catch_planted_mistake(mutate):
     m = _fresh_oracle()
