@@ -139,3 +139,51 @@ def prefill_case(L: int, H: int, d: int, dtype: str, seed: int, device: str = "c
     K = normal((L, H, d), seed * 11 + 2, dtype, device)
     V = normal((L, H, d), seed * 11 + 3, dtype, device)
     return Q, K, V
+
+
+# ---------------------------------------------------------------- spike inputs
+#
+# A query set to a multiple of one key makes that key's score stand far above
+# every other score, so the attention output is (almost exactly) that key's
+# value row when the key is visible, and something else entirely when it is
+# not.  Placing the key on an edge of the visible set turns a one-key error in
+# the mask into an O(1) error in the output.  Which (query, key) pairs sit on
+# an edge is decided by the caller; these functions only copy rows.
+
+SPIKE_GAIN = 4.0
+
+
+def spike_packed_queries(Q: torch.Tensor, K: torch.Tensor, probes, gain: float = SPIKE_GAIN) -> torch.Tensor:
+    """Copy of Q ([L, H, d]) where, for each (row, key) in ``probes``
+    (0-based packed rows, distinct rows), Q[row, h] = gain * K[key, h] for
+    every head h, rounded to Q's dtype."""
+    Q = Q.clone()
+    rows = [int(r) for r, _ in probes]
+    if len(set(rows)) != len(rows):
+        raise ValueError("one probe per query row")
+    if probes:
+        r = torch.tensor(rows, device=Q.device)
+        k = torch.tensor([int(j) for _, j in probes], device=Q.device)
+        Q[r] = (K[k].to(torch.float32) * gain).to(Q.dtype)
+    return Q
+
+
+def history_key(case: DecodeCase, b: int, pos: int) -> torch.Tensor:
+    """Key [H, d] at 1-based logical position ``pos`` of sequence b: the
+    reference rows 1..L_m[b], then output j at position L_m[b] + j."""
+    L = case.ref_lens[b]
+    if 1 <= pos <= L:
+        return case.K_ref[b, :, pos - 1]
+    j = pos - L
+    if not 1 <= j <= case.T:
+        raise ValueError("position outside the generated history")
+    return case.k[j - 1, b]
+
+
+def spike_decode_queries(case: DecodeCase, probes, gain: float = SPIKE_GAIN) -> None:
+    """In place: for each (t, b, pos) in ``probes``, the query of decode step
+    t (``case.q[t-1, b]``) becomes gain * (key at logical position pos of
+    sequence b), for every head, rounded to the case's dtype."""
+    for t, b, pos in probes:
+        key = history_key(case, int(b), int(pos)).to(torch.float32)
+        case.q[int(t) - 1, int(b)] = (key * gain).to(case.q.dtype)
