@@ -126,6 +126,22 @@ rswa_status rswa_init(rswa_handle* out, rswa_mode mode, int L_m_cap, int n, int 
 rswa_status rswa_load_reference(rswa_handle h, const void* K_ref, const void* V_ref,
                                 int ref_stride, const int32_t* ref_lens);
 
+/* Appends one chunk of the reference segment after the rows already loaded,
+ * so a reference can be written as it is produced (for example page by page,
+ * 256 vision tokens each) and still be "encoded once and never updated":
+ * every row is written once, at its final cache row.  A handle starts with
+ * an empty reference; rswa_load_reference replaces it, chunks extend it.
+ *   K, V: device [batch][H][chunk_stride][d]; rows [0, rows[b]) of sequence
+ *     b's chunk become its reference rows L_m[b] .. L_m[b] + rows[b] - 1.
+ *   rows: HOST int32[batch], 0 <= rows[b] <= chunk_stride and the total
+ *     L_m[b] + rows[b] <= L_m_cap (else RSWA_ERR_CAPACITY, nothing enqueued).
+ * Only while no output has been appended (T = 0; else RSWA_ERR_STATE: the
+ * output ring starts right after the reference rows).  Sets T = 0.  Decode
+ * calls need every sequence to hold at least one reference row.  The result
+ * is the cache rswa_load_reference leaves for the concatenated chunks. */
+rswa_status rswa_load_reference_chunk(rswa_handle h, const void* K, const void* V, int chunk_stride,
+                                      const int32_t* rows);
+
 /* Fills the cache from the packed (teacher-forced) layout, so decoding can
  * continue after a prefill: the result is the cache that
  * rswa_load_reference followed by T0 appends would leave.  The reference
@@ -168,6 +184,21 @@ rswa_status rswa_decode(rswa_handle h, const void* q, void* o, float scale);
  * such limit (its plan covers the whole ring). */
 rswa_status rswa_append_decode(rswa_handle h, const void* k, const void* v,
                                const void* q, void* o, float scale);
+
+/* One decode step of an R-layer decoder: rswa_append_decode for layers
+ * 0 .. R-1 in order, one kernel each, on the handles' common stream (the
+ * handles of one model's attention layers).  Layer r's kernel may start
+ * copying its reference rows while layer r-1 still runs (programmatic
+ * dependent launch); it reads q, k, v and its ring after layer r-1 has
+ * finished.
+ *   hs: HOST array of R distinct handles on one device and one stream.
+ *   k, v, q, o: HOST arrays of R device pointers, each [batch_r][H_r][d_r] of
+ *     its handle.
+ * Every argument and every handle's state is checked before the first launch
+ * (errors enqueue nothing); a CUDA launch error stops at that layer.  A
+ * captured CUDA graph of this call replays whole decode steps. */
+rswa_status rswa_append_decode_layers(const rswa_handle* hs, int R, const void* const* k, const void* const* v,
+                                      const void* const* q, void* const* o, float scale);
 
 /* Synchronous: cache occupancy L_m[b] + min(n, T[b]) (FULL: L_m[b] + T[b])
  * per sequence, Eq.(6) / Eq.(5).  out: HOST int32[batch]. */
@@ -250,9 +281,9 @@ rswa_status rswa_masked_forward_varlen(const void* Q, const void* K, const void*
 /* ------------------------------------------------------------------------
  * Decode without allocation.  The pages have no counterpart to this call;
  * it exists for callers that cannot allocate device memory: a plugin inside
- * a host framework that owns every device allocation, code that must avoid
- * the implicitly synchronising cudaMalloc / cudaFree, or code running while
- * a stream is being captured, where allocation calls are not permitted.
+ * a host framework whose own allocator owns every device allocation (memory
+ * taken behind its back breaks its accounting), or code that must avoid the
+ * implicitly synchronising cudaMalloc / cudaFree on a latency-critical path.
  *
  * One-shot decode attention over caller-owned caches, with no handle and no
  * workspace: the kernel's scratch (launch plan, split-K partials, tickets)
@@ -266,16 +297,23 @@ rswa_status rswa_masked_forward_varlen(const void* Q, const void* K, const void*
  *   q, o: device [batch][H][d].  scale <= 0 selects 1/sqrt(d).
  * Limits: batch * H <= 1024; d = 64 or 128.  Larger sizes return
  * RSWA_ERR_CAPACITY with a message in rswa_last_error().
- * The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture.  Every call reuses the same array and clears
- * what must start at zero, so calls whose kernels overlap on the GPU race:
- * order them on one stream.  Kernel-side error flags are not reported.
+ * The first call on a device (and the first after that device's context was
+ * reset) looks up the array's device address (cudaGetSymbolAddress) with
+ * that device current.  Every call reuses the same array and clears what
+ * must start at zero, so calls whose kernels overlap on the GPU race: order
+ * them on one stream.  The plan is staged with stream-ordered copies from
+ * host memory.
  * ---------------------------------------------------------------------- */
 rswa_status rswa_decode_noalloc(const void* k_cache, const void* v_cache, int S_cap,
                                 const int32_t* cache_lens, const void* q, void* o,
                                 int batch, int H, int d, rswa_dtype dtype, float scale,
                                 void* stream);
+
+/* Synchronous (waits for `stream`): RSWA_ERR_DEVICE if a decode launched by
+ * rswa_decode_noalloc on the current device raised the device error word (a
+ * bounded wait that timed out) since the last check; the word is then
+ * cleared.  Allocates nothing. */
+rswa_status rswa_decode_noalloc_check(void* stream);
 
 /* ------------------------------------------------------------------------
  * Introspection (host only; needs no device).

@@ -23,7 +23,7 @@ import torch
 from . import _native
 from ._native import MODE_FULL, MODE_RSWA, RSWAError, check
 
-__all__ = ["RSWA", "masked_forward", "masked_forward_varlen", "RSWAError", "MODE_RSWA", "MODE_FULL", "library_version"]
+__all__ = ["RSWA", "append_decode_layers", "masked_forward", "masked_forward_varlen", "RSWAError", "MODE_RSWA", "MODE_FULL", "library_version"]
 
 _DT = {torch.float32: _native.F32, torch.bfloat16: _native.BF16}
 
@@ -155,6 +155,21 @@ class RSWA:
         self._sync_stream()
         check(_native.lib().rswa_load_packed(self._h, K.data_ptr(), V.data_ptr(), L, lens, int(T0)))
 
+    def load_reference_chunk(self, K: torch.Tensor, V: torch.Tensor, rows: Sequence[int]) -> None:
+        """Appends rows [0, rows[b]) of K, V ([B, H, stride, d] on the device)
+        to sequence b's reference, after the rows already loaded; only
+        before the first output is appended."""
+        if K.dim() != 4:
+            raise ValueError("K must be [B, H, stride, d]")
+        stride = K.shape[2]
+        _check_tensor("K", K, (self.batch, self.H, stride, self.d), self.dtype, self.device)
+        _check_tensor("V", V, (self.batch, self.H, stride, self.d), self.dtype, self.device)
+        if len(rows) != self.batch:
+            raise ValueError("rows must have one entry per sequence")
+        r = (C.c_int32 * self.batch)(*[int(x) for x in rows])
+        self._sync_stream()
+        check(_native.lib().rswa_load_reference_chunk(self._h, K.data_ptr(), V.data_ptr(), stride, r))
+
     def append(self, k: torch.Tensor, v: torch.Tensor) -> None:
         self._vec("k", k)
         self._vec("v", v)
@@ -209,6 +224,30 @@ class RSWA:
         """Raises RSWAError if a kernel flagged a device-side error."""
         self._sync_stream()
         check(_native.lib().rswa_check(self._h))
+
+
+def append_decode_layers(layers: Sequence[RSWA], k: Sequence[torch.Tensor], v: Sequence[torch.Tensor],
+                         q: Sequence[torch.Tensor], out: Optional[Sequence[torch.Tensor]] = None,
+                         scale: float = 0.0) -> list:
+    """One decode step of an R-layer decoder: append_decode on every layer
+    handle in order (one C call, one kernel per layer).  k[r], v[r], q[r],
+    out[r]: [B, H, d] tensors of layer r's handle.  Returns the outputs."""
+    R = len(layers)
+    if not (len(k) == len(v) == len(q) == R) or (out is not None and len(out) != R):
+        raise ValueError("one k, v, q (and out) per layer")
+    outs = [torch.empty_like(q[r]) for r in range(R)] if out is None else list(out)
+    for r, a in enumerate(layers):
+        a._vec("k", k[r])
+        a._vec("v", v[r])
+        a._vec("q", q[r])
+        a._vec("out", outs[r])
+        a._sync_stream()
+    P = C.c_void_p * R
+    hs = P(*[a._h.value for a in layers])
+    check(_native.lib().rswa_append_decode_layers(
+        hs, R, P(*[t.data_ptr() for t in k]), P(*[t.data_ptr() for t in v]), P(*[t.data_ptr() for t in q]),
+        P(*[t.data_ptr() for t in outs]), float(scale)))
+    return outs
 
 
 def masked_forward(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, L_m: int, n: int,

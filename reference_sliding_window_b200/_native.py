@@ -26,9 +26,12 @@ _PROTOS = {
     "rswa_init": (_i, [C.POINTER(_p), _i, _i, _i, _i, _i, _i, _i, _i, _p, _p, _p, _sz, _p]),
     "rswa_load_reference": (_i, [_p, _p, _p, _i, C.POINTER(C.c_int32)]),
     "rswa_load_packed": (_i, [_p, _p, _p, _i, C.POINTER(C.c_int32), _i]),
+    "rswa_load_reference_chunk": (_i, [_p, _p, _p, _i, C.POINTER(C.c_int32)]),
     "rswa_append": (_i, [_p, _p, _p]),
     "rswa_decode": (_i, [_p, _p, _p, _f]),
     "rswa_append_decode": (_i, [_p, _p, _p, _p, _p, _f]),
+    "rswa_append_decode_layers": (_i, [C.POINTER(_p), _i, C.POINTER(_p), C.POINTER(_p), C.POINTER(_p),
+                                      C.POINTER(_p), _f]),
     "rswa_cache_len": (_i, [_p, C.POINTER(C.c_int32)]),
     "rswa_step_count": (_i, [_p, C.POINTER(C.c_int32)]),
     "rswa_cache_positions": (_i, [_p, _i, C.POINTER(C.c_int64), _i, C.POINTER(_i)]),
@@ -41,6 +44,7 @@ _PROTOS = {
     "rswa_masked_forward_varlen": (_i, [_p, _p, _p, _p, C.POINTER(C.c_int32), C.POINTER(C.c_int32), _i, _i,
                                        _i, _i, _i, _f, _i, _p]),
     "rswa_decode_noalloc": (_i, [_p, _p, _i, C.POINTER(C.c_int32), _p, _p, _i, _i, _i, _i, _f, _p]),
+    "rswa_decode_noalloc_check": (_i, [_p]),
     "rswa_plan_decode": (_i, [_i, _i, C.POINTER(C.c_int32), _i, _i, _i, _i, C.POINTER(C.c_int32), _i,
                               C.POINTER(C.c_int32), _i, C.POINTER(_i), C.POINTER(_i), C.POINTER(_i)]),
     "rswa_last_error": (C.c_char_p, []),

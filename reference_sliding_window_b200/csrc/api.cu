@@ -3,6 +3,7 @@
 // kernel launches.  Host code only; every step of the attention runs in the
 // kernels of decode.cu, append.cu and the masked-forward files.
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdarg.h>
@@ -11,6 +12,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -58,6 +60,22 @@ static bool dtype_ok(rswa_dtype t) { return t == RSWA_F32 || t == RSWA_BF16; }
 
 namespace rswa {
 
+unsigned long long current_context_id() {
+  typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+  static CtxGetIdFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetIdFn>(ptr);
+  });
+  unsigned long long id = 0;
+  if (!fn || fn(nullptr, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Split-K partials are bounded: a span plan has at most one item per slab
@@ -73,6 +91,8 @@ WorkspaceLayout workspace_layout(int B, int H, int d) {
   w.T = off;
   off = align_up(off + 4, 256);
   w.Lm = off;
+  off = align_up(off + 4 * (size_t)B, 256);
+  w.chunk = off;
   off = align_up(off + 4 * (size_t)B, 256);
   w.tickets = off;
   off = align_up(off + 4 * (size_t)B * H, 256);
@@ -177,7 +197,9 @@ static void make_plan(rswa_ctx* c) {
     c->n_ctas = Gc;
     return;
   }
-  const int G = (int)std::min<long long>(std::min(c->num_sms, c->lay.max_ctas), total);
+  // At most kMinMergeCap / 2 CTAs, so a slab never has more partials than one
+  // CTA can merge (two slabs at a time) in shared memory.
+  const int G = (int)std::min<long long>(std::min(std::min(c->num_sms, c->lay.max_ctas), kMinMergeCap / 2), total);
   c->items.clear();
   c->cta_begin.assign(G + 1, 0);
   std::vector<int> first_item(nbh, -1), count(nbh, 0);
@@ -410,6 +432,61 @@ extern "C" rswa_status rswa_load_reference(rswa_handle h, const void* K_ref, con
   return RSWA_OK;
 }
 
+extern "C" rswa_status rswa_load_reference_chunk(rswa_handle h, const void* K, const void* V, int chunk_stride,
+                                                 const int32_t* rows) {
+  if (rswa_status st = check_handle(h)) return st;
+  if (!K || !V || !rows) return fail(RSWA_ERR_ARG, "rswa_load_reference_chunk: null argument");
+  if (!aligned16(K) || !aligned16(V))
+    return fail(RSWA_ERR_ARG, "rswa_load_reference_chunk: K/V must be 16-byte aligned");
+  if (chunk_stride < 1) return fail(RSWA_ERR_ARG, "rswa_load_reference_chunk: chunk_stride=%d", chunk_stride);
+  if (h->T_host != 0)
+    return fail(RSWA_ERR_STATE, "rswa_load_reference_chunk: outputs were appended; the reference is complete "
+                                "(rswa_reset first)");
+  std::vector<int32_t> Lm(h->B, 0);
+  if (h->Lm.size() == (size_t)h->B) Lm = h->Lm;
+  int max_rows = 0;
+  for (int b = 0; b < h->B; ++b) {
+    const int r = rows[b];
+    if (r < 0 || r > chunk_stride || (long long)Lm[b] + r > h->L_m_cap)
+      return fail(RSWA_ERR_CAPACITY,
+                  "rswa_load_reference_chunk: rows[%d]=%d outside [0, chunk_stride=%d] or past L_m_cap=%d "
+                  "(%d rows loaded)", b, r, chunk_stride, h->L_m_cap, Lm[b]);
+    Lm[b] += r;
+    max_rows = std::max(max_rows, r);
+  }
+  if (rswa_status st = use_device(h)) return st;
+  h->Lm = Lm;
+  bool all = true;
+  for (int b = 0; b < h->B; ++b) all = all && Lm[b] >= 1;
+  RSWA_CUDA(cudaMemcpyAsync(h->ws + h->lay.Lm, h->Lm.data(), 4 * (size_t)h->B, cudaMemcpyHostToDevice,
+                            h->stream),
+            "upload reference lengths");
+  RSWA_CUDA(cudaMemcpyAsync(h->ws + h->lay.chunk, rows, 4 * (size_t)h->B, cudaMemcpyHostToDevice, h->stream),
+            "upload chunk rows");
+  RSWA_CUDA(cudaMemsetAsync(h->ws + h->lay.T, 0, 4, h->stream), "reset step counter");
+  if (all) {
+    h->plan_window = h->mode == RSWA_MODE_RSWA ? h->n : std::min(h->T_cap, 64);
+    make_plan(h);
+    if (rswa_status st = upload_plan(h)) return st;
+  }
+  LoadChunkParams p;
+  p.kc = h->kc;
+  p.vc = h->vc;
+  p.K = K;
+  p.V = V;
+  p.B = h->B;
+  p.H = h->H;
+  p.S_cap = h->S_cap;
+  p.row_bytes = h->row_bytes;
+  p.chunk_stride = chunk_stride;
+  p.Lm = ws_i32(h, h->lay.Lm);
+  p.rows = ws_i32(h, h->lay.chunk);
+  if (max_rows > 0) RSWA_CUDA(launch_load_chunk(p, max_rows, h->stream), "load_chunk kernel");
+  // Decoding needs every sequence's reference to be non-empty.
+  h->loaded = all;
+  return RSWA_OK;
+}
+
 extern "C" rswa_status rswa_load_packed(rswa_handle h, const void* K, const void* V, int seq_stride,
                                         const int32_t* ref_lens, int T0) {
   if (rswa_status st = check_handle(h)) return st;
@@ -462,7 +539,9 @@ extern "C" rswa_status rswa_load_packed(rswa_handle h, const void* K, const void
 // ------------------------------------------------------------------- steps
 
 static rswa_status check_step(rswa_ctx* c, bool appending, const char* who) {
-  if (!c->loaded) return fail(RSWA_ERR_STATE, "%s: call rswa_load_reference first", who);
+  if (!c->loaded)
+    return fail(RSWA_ERR_STATE, "%s: no reference loaded (rswa_load_reference, rswa_load_packed, or "
+                                "rswa_load_reference_chunk until every sequence has a row)", who);
   if (appending && c->mode == RSWA_MODE_FULL && c->T_host + 1 > c->T_cap)
     return fail(RSWA_ERR_CAPACITY, "%s: FULL mode holds at most T_cap=%d outputs", who, c->T_cap);
   return RSWA_OK;
@@ -566,6 +645,31 @@ extern "C" rswa_status rswa_append_decode(rswa_handle h, const void* k, const vo
                                           void* o, float scale) {
   if (rswa_status st = check_handle(h)) return st;
   return run_decode(h, k, v, q, o, scale, true, "rswa_append_decode");
+}
+
+extern "C" rswa_status rswa_append_decode_layers(const rswa_handle* hs, int R, const void* const* k,
+                                                 const void* const* v, const void* const* q, void* const* o,
+                                                 float scale) {
+  static const char* who = "rswa_append_decode_layers";
+  if (!hs || !k || !v || !q || !o) return fail(RSWA_ERR_ARG, "%s: null argument", who);
+  if (R < 1) return fail(RSWA_ERR_ARG, "%s: R=%d layers", who, R);
+  if (!(scale == scale) || isinf(scale)) return fail(RSWA_ERR_ARG, "%s: scale is not finite", who);
+  // Everything is checked before the first launch.
+  for (int r = 0; r < R; ++r) {
+    rswa_ctx* c = hs[r];
+    if (!c) return fail(RSWA_ERR_ARG, "%s: handle %d is null", who, r);
+    if (!k[r] || !v[r] || !q[r] || !o[r]) return fail(RSWA_ERR_ARG, "%s: null tensor for layer %d", who, r);
+    if (!aligned16(k[r]) || !aligned16(v[r]) || !aligned16(q[r]) || !aligned16(o[r]))
+      return fail(RSWA_ERR_ARG, "%s: tensors of layer %d must be 16-byte aligned", who, r);
+    if (c->device != hs[0]->device || c->stream != hs[0]->stream)
+      return fail(RSWA_ERR_ARG, "%s: layer %d is on another device or stream than layer 0", who, r);
+    for (int r2 = 0; r2 < r; ++r2)
+      if (hs[r2] == c) return fail(RSWA_ERR_ARG, "%s: handle of layer %d repeats layer %d", who, r, r2);
+    if (rswa_status st = check_step(c, true, who)) return st;
+  }
+  for (int r = 0; r < R; ++r)
+    if (rswa_status st = run_decode(hs[r], k[r], v[r], q[r], o[r], scale, true, who)) return st;
+  return RSWA_OK;
 }
 
 // ----------------------------------------------------------------- queries

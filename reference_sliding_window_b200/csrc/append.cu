@@ -112,6 +112,40 @@ __global__ void __launch_bounds__(256) load_packed_kernel(const __grid_constant_
   __threadfence();
 }
 
+// grid.y = B*H slabs: appends one chunk of reference rows after the rows
+// already loaded ("encoded once": a reference can arrive page by page, each
+// page's rows written once and never again).
+__global__ void __launch_bounds__(256) load_chunk_kernel(const __grid_constant__ LoadChunkParams p) {
+  const int bh = blockIdx.y;
+  const int b = bh / p.H;
+  const int rows = p.rows[b];
+  const int dst0 = p.Lm[b] - rows;
+  const int vpr = p.row_bytes / 16;
+  const long long n_vec = (long long)rows * vpr;
+  const uint8_t* ks = static_cast<const uint8_t*>(p.K) + (size_t)bh * p.chunk_stride * p.row_bytes;
+  const uint8_t* vs = static_cast<const uint8_t*>(p.V) + (size_t)bh * p.chunk_stride * p.row_bytes;
+  uint8_t* kd = static_cast<uint8_t*>(p.kc) + ((size_t)bh * p.S_cap + dst0) * p.row_bytes;
+  uint8_t* vd = static_cast<uint8_t*>(p.vc) + ((size_t)bh * p.S_cap + dst0) * p.row_bytes;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n_vec;
+       i += (long long)gridDim.x * blockDim.x) {
+    *reinterpret_cast<uint4*>(kd + i * 16) = *reinterpret_cast<const uint4*>(ks + i * 16);
+    *reinterpret_cast<uint4*>(vd + i * 16) = *reinterpret_cast<const uint4*>(vs + i * 16);
+  }
+  // Same contract as load_reference_kernel: decode kernels may copy
+  // reference rows before their dependency wait.
+  __threadfence();
+}
+
+cudaError_t launch_load_chunk(const LoadChunkParams& p, int max_rows, cudaStream_t stream) {
+  const long long vecs = (long long)max_rows * (p.row_bytes / 16);
+  long long gx = (vecs + 255) / 256;
+  if (gx > 1024) gx = 1024;
+  if (gx < 1) gx = 1;
+  dim3 grid((unsigned)gx, (unsigned)(p.B * p.H));
+  load_chunk_kernel<<<grid, 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_append(const AppendParams& p, cudaStream_t stream) {
   append_kernel<<<1, 256, 0, stream>>>(p);
   return cudaGetLastError();

@@ -22,4 +22,18 @@ struct LoadPackedParams {
 };
 cudaError_t launch_load_packed(const LoadPackedParams& p, int max_rows, cudaStream_t stream);
 
+// One chunk of the reference segment: rows [0, rows[b]) of sequence b's chunk
+// (K/V laid out [B][H][chunk_stride][d]) go to cache rows
+// [Lm[b] - rows[b], Lm[b]) of its slabs, Lm already counting the chunk.
+struct LoadChunkParams {
+  void* kc;
+  void* vc;
+  const void* K;
+  const void* V;
+  int B, H, S_cap, row_bytes, chunk_stride;
+  const int32_t* Lm;    // device [B], after the chunk
+  const int32_t* rows;  // device [B]
+};
+cudaError_t launch_load_chunk(const LoadChunkParams& p, int max_rows, cudaStream_t stream);
+
 }  // namespace rswa

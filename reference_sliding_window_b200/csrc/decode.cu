@@ -218,14 +218,12 @@ __device__ __forceinline__ int valid_rows(const DecodeParams& p, int Lm, int T_n
   return min(len, p.S_cap);
 }
 
-// Log-sum-exp merge of the nparts partials of one slab into its output row.
-// A slab's partials are contiguous, so all consumer threads copy them into
-// shared memory (the stage ring, idle by then) with independent 16-byte
-// loads in one round, then thread `dim` folds them there.  Chunks of
-// `cap` partials bound the shared memory used.
-// The same for the slabs of up to two items at once (their partials together
-// fit in the buffer): one round of loads for both, then thread x*D + dim
-// folds item x.
+// Log-sum-exp merge of the partials of up to two slabs into their output
+// rows.  A slab's partials are contiguous, so all consumer threads copy both
+// slabs' partials into shared memory (the stage ring, idle by then) with
+// independent 16-byte loads in one round, then thread x*D + dim folds item x.
+// The host planner keeps a slab within kMergeCap / 2 partials, so two always
+// fit.
 template <typename T, int D, int NT>
 __device__ __forceinline__ void merge_partials_joint(const DecodeParams& p, const DecodeItem& i0,
                                                      const DecodeItem& i1, int n_its, int tid, float* buf) {
@@ -262,47 +260,6 @@ __device__ __forceinline__ void merge_partials_joint(const DecodeParams& p, cons
     store_elem(static_cast<T*>(p.o) + (size_t)(x ? i1.bh : i0.bh) * D + dd, acc / L);
   }
   named_barrier_sync(1, NT);
-}
-
-template <typename T, int D, int NT>
-__device__ __forceinline__ void merge_partials(const DecodeParams& p, const DecodeItem& item, int tid,
-                                               float* buf, int cap) {
-  constexpr int RW = D + 4;  // floats per partial: o[D], m, l, pad
-  const float4* src = reinterpret_cast<const float4*>(p.partials + (size_t)item.part_first * RW);
-  float M_run = -INFINITY, L_run = 0.f, o_run = 0.f;
-  for (int c0 = 0; c0 < item.nparts; c0 += cap) {
-    const int cn = min(cap, item.nparts - c0);
-    const int nvec = cn * RW / 4;
-    float4* dst = reinterpret_cast<float4*>(buf);
-    const float4* s0 = src + (size_t)c0 * RW / 4;
-    // independent loads, issued together: one L2 round trip per 4*NT vectors
-    for (int i = tid; i < nvec; i += 4 * NT) {
-      float4 v[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if (i + u * NT < nvec) v[u] = __ldcg(s0 + i + u * NT);
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if (i + u * NT < nvec) dst[i + u * NT] = v[u];
-    }
-    named_barrier_sync(1, NT);
-    if (tid < D) {
-      float Mc = M_run;
-      for (int i = 0; i < cn; ++i) Mc = fmaxf(Mc, buf[i * RW + D]);  // finite: the slab has rows
-      const float a = exp2f(M_run - Mc);  // 0 on the first chunk
-      float acc = 0.f, Lc = 0.f;
-      for (int i = 0; i < cn; ++i) {
-        const float w = exp2f(buf[i * RW + D] - Mc);  // exp2(-inf) = 0 for empty partials
-        acc = fmaf(w, buf[i * RW + tid], acc);
-        Lc = fmaf(w, buf[i * RW + D + 1], Lc);
-      }
-      o_run = o_run * a + acc;
-      L_run = L_run * a + Lc;
-      M_run = Mc;
-    }
-    named_barrier_sync(1, NT);  // buf is reused by the next chunk
-  }
-  if (tid < D) store_elem(static_cast<T*>(p.o) + (size_t)item.bh * D + tid, o_run / L_run);
 }
 
 template <typename T, int D, bool APPEND>
@@ -791,11 +748,11 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
     if (nm > 0) {
       const DecodeItem m0 = item_at(f0 ? pend0 : pend1);
       const DecodeItem m1 = item_at(pend1 >= 0 ? pend1 : pend0);
+      // The host planner keeps every slab within kMergeCap / 2 partials.
       if (m0.nparts + (nm > 1 ? m1.nparts : 0) <= Tr::kMergeCap) {
         merge_partials_joint<T, D, NT>(p, m0, m1, nm, tid, merge_buf);
-      } else {
-        merge_partials<T, D, NT>(p, m0, tid, merge_buf, Tr::kMergeCap);
-        if (nm > 1) merge_partials<T, D, NT>(p, m1, tid, merge_buf, Tr::kMergeCap);
+      } else if (tid == 0) {
+        flag_error(p.err, kErrPlanShort);
       }
       if (tid == 0) {
         RSWA_STAMP(13);
@@ -818,17 +775,12 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
 template <typename T, int D, bool A>
 static cudaError_t launch_one(const DecodeParams& p, int grid, cudaStream_t stream) {
   using Tr = DecTraits<T, D>;
-  static bool configured[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<T, D, A>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)Tr::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    configured[dev] = true;
-  }
+  static PerContextOnce attr_once;
+  cudaError_t e = attr_once.run([] {
+    return cudaFuncSetAttribute(decode_kernel<T, D, A>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)Tr::kSmemBytes);
+  });
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(Tr::kThreads);
@@ -892,6 +844,11 @@ cudaError_t launch_decode(int elem, int D, bool append, const DecodeParams& p, i
   if (elem == kF32 && D == 64) return launch_d<float, 64>(append, p, grid, stream);
   return cudaErrorInvalidValue;
 }
+
+static_assert(DecTraits<__nv_bfloat16, 128>::kMergeCap >= kMinMergeCap &&
+                  DecTraits<__nv_bfloat16, 64>::kMergeCap >= kMinMergeCap &&
+                  DecTraits<float, 128>::kMergeCap >= kMinMergeCap && DecTraits<float, 64>::kMergeCap >= kMinMergeCap,
+              "the planners' CTA cap assumes every variant merges kMinMergeCap partials");
 
 size_t decode_smem_bytes(int elem, int D) {
   if (elem == kBF16 && D == 128) return DecTraits<__nv_bfloat16, 128>::kSmemBytes;

@@ -5,7 +5,40 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <mutex>
+
 namespace rswa {
+
+// Identity of the calling thread's current CUDA context (cuCtxGetId: never
+// reused within a process, so a context created after a device reset gets a
+// new one), or 0 if none is current or the driver does not provide it.
+unsigned long long current_context_id();
+
+// Host set-up that must run once per CUDA context of a device (a kernel's
+// shared-memory attribute, a symbol's device address), thread-safe.  run()
+// calls f() unless it already succeeded in the current context of the
+// current device.
+class PerContextOnce {
+ public:
+  template <typename F>
+  cudaError_t run(F&& f) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu_);
+    const unsigned long long id = current_context_id();
+    if (id != 0 && done_[dev] == id) return cudaSuccess;
+    e = f();
+    if (e == cudaSuccess) done_[dev] = id != 0 ? id : current_context_id();
+    return e;
+  }
+
+ private:
+  static constexpr int kMaxDevices = 64;
+  std::mutex mu_;
+  unsigned long long done_[kMaxDevices] = {};
+};
 
 // Bits of the device error word (workspace).  Kernels set them with atomicOr
 // and return; they never trap.
@@ -38,6 +71,7 @@ struct WorkspaceLayout {
   size_t done;       // int32: end-of-launch ticket (fused append+decode)
   size_t T;          // int32: outputs appended so far (every sequence advances together)
   size_t Lm;         // int32[B]: reference rows
+  size_t chunk;      // int32[B]: rows of the reference chunk being appended
   size_t tickets;    // int32[B*H]: split-K tickets
   size_t items;      // DecodeItem[items_cap]
   size_t cta_begin;  // int32[max_ctas + 1]: first item of each CTA
@@ -91,6 +125,10 @@ cudaError_t launch_decode(int elem, int D, bool append, const DecodeParams& p, i
                           cudaStream_t stream);
 // Dynamic shared memory the decode kernel needs for (elem, D).
 size_t decode_smem_bytes(int elem, int D);
+// Split-K partials the decode kernel can merge in shared memory for two slabs
+// at once, for every (elem, D) it supports (checked in decode.cu).  The
+// planners use at most kMinMergeCap / 2 CTAs, so a slab never has more.
+constexpr int kMinMergeCap = 372;
 
 struct AppendParams {
   void* kc;

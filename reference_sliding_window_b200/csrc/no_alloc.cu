@@ -1,21 +1,25 @@
 // rswa_decode_noalloc: one-shot decode attention that allocates nothing.
 //
 // Some callers cannot allocate device memory: a plugin running inside a host
-// framework that owns every device allocation, code that must not make the
-// implicitly synchronising cudaMalloc / cudaFree calls on a latency-critical
-// path, or code that runs while a stream is being captured, where allocation
-// calls are not permitted.  The handle API needs a caller-provided workspace;
-// this entry point instead keeps the decode kernel's scratch (launch plan,
-// split-K partials, tickets, counters) in one file-scope device array that
-// every device loading the library holds until the process exits.
+// framework that owns every device allocation (its allocator hands out all
+// memory, and a library that called cudaMalloc behind its back would break
+// its accounting), or code that must not make the implicitly synchronising
+// cudaMalloc / cudaFree calls on a latency-critical path.  The handle API
+// needs a caller-provided workspace; this entry point instead keeps the
+// decode kernel's scratch (launch plan, split-K partials, tickets, counters)
+// in one file-scope device array that every device loading the library holds
+// until the process exits.
 //
 // The caller passes the caches, the query and the output.  Every call reuses
 // the same array, so two calls whose kernels overlap on the GPU race; issue
 // them on one stream (or otherwise order them).  The parts that must start at
-// zero are cleared by every call.
+// zero (launch ticket, step counter, split-K tickets) are cleared by every
+// call; the device error word is kept until rswa_decode_noalloc_check reads
+// and clears it.
 
 #include <cuda_runtime.h>
 #include <math.h>
+#include <stdio.h>
 
 #include <algorithm>
 #include <mutex>
@@ -44,10 +48,17 @@ constexpr size_t kNaBytes = kNaPartials + 4ull * (kNoAllocMaxD + 4) * kNoAllocMa
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNaBytes];
 
-// Device address of the scratch, resolved once per device (host code may not
-// use the symbol itself as a device pointer).
+// Device address of the scratch in the current context of each device.  Host
+// code may not use the symbol itself as a device pointer (it names a host-side
+// stand-in), so the address is looked up with cudaGetSymbolAddress, with the
+// device current, on the first call in each context: a context made after a
+// device reset loads the module again and gets its own copy of the array.
 constexpr int kMaxDevices = 64;
-static void* g_scratch_addr[kMaxDevices];
+struct ScratchAddr {
+  unsigned long long ctx;
+  void* ptr;
+};
+static ScratchAddr g_scratch_addr[kMaxDevices];
 static std::mutex g_scratch_mu;
 
 static cudaError_t scratch_for_current_device(uint8_t** out) {
@@ -56,13 +67,16 @@ static cudaError_t scratch_for_current_device(uint8_t** out) {
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
+  const unsigned long long ctx = current_context_id();
+  ScratchAddr& a = g_scratch_addr[dev];
+  if (ctx == 0 || a.ctx != ctx || !a.ptr) {
     void* ptr = nullptr;
     e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
     if (e != cudaSuccess) return e;
-    g_scratch_addr[dev] = ptr;
+    a.ptr = ptr;
+    a.ctx = ctx != 0 ? ctx : current_context_id();
   }
-  *out = static_cast<uint8_t*>(g_scratch_addr[dev]);
+  *out = static_cast<uint8_t*>(a.ptr);
   return cudaSuccess;
 }
 
@@ -113,7 +127,7 @@ extern "C" rswa_status rswa_decode_noalloc(const void* k_cache, const void* v_ca
   const int nbh = batch * H;
   long long total = 0;
   for (int bh = 0; bh < nbh; ++bh) total += (g_na_lens[bh / H] + 31) / 32;
-  const int G = (int)std::min<long long>(std::min(sms, kNoAllocMaxCtas), total);
+  const int G = (int)std::min<long long>(std::min(std::min(sms, kNoAllocMaxCtas), kMinMergeCap / 2), total);
   int n_items = 0, bh = 0, st = 0;
   int first_item = 0;
   for (int g = 0; g < G; ++g) {
@@ -146,8 +160,9 @@ extern "C" rswa_status rswa_decode_noalloc(const void* k_cache, const void* v_ca
   g_na_begin[G] = n_items;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // Counters and tickets must start at zero; plan and lengths are uploaded.
-  if (cudaMemsetAsync(scratch, 0, kNaLm, s) != cudaSuccess ||
+  // Counters and tickets must start at zero (the error word is kept for
+  // rswa_decode_noalloc_check); plan and lengths are uploaded.
+  if (cudaMemsetAsync(scratch + kNaDone, 0, kNaLm - kNaDone, s) != cudaSuccess ||
       cudaMemsetAsync(scratch + kNaTickets, 0, 4 * (size_t)nbh, s) != cudaSuccess ||
       cudaMemcpyAsync(scratch + kNaLm, g_na_lens, 4 * (size_t)batch, cudaMemcpyHostToDevice, s) != cudaSuccess ||
       cudaMemcpyAsync(scratch + kNaItems, g_na_items, sizeof(DecodeItem) * n_items, cudaMemcpyHostToDevice, s) !=
@@ -183,4 +198,23 @@ extern "C" rswa_status rswa_decode_noalloc(const void* k_cache, const void* v_ca
   if (launch_decode(dtype == RSWA_BF16 ? kBF16 : kF32, d, false, p, G, s) != cudaSuccess)
     return na_fail(RSWA_ERR_CUDA, "decode kernel launch failed");
   return RSWA_OK;
+}
+
+extern "C" rswa_status rswa_decode_noalloc_check(void* stream) {
+  uint8_t* scratch = nullptr;
+  if (scratch_for_current_device(&scratch) != cudaSuccess)
+    return na_fail(RSWA_ERR_CUDA, "cudaGetSymbolAddress of the static scratch failed");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t err = 0;
+  if (cudaMemcpyAsync(&err, scratch + kNaErr, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return na_fail(RSWA_ERR_CUDA, "reading the device error word failed");
+  if (err == 0) return RSWA_OK;
+  if (cudaMemsetAsync(scratch + kNaErr, 0, 4, s) != cudaSuccess)
+    return na_fail(RSWA_ERR_CUDA, "clearing the device error word failed");
+  char msg[96];
+  snprintf(msg, sizeof(msg), "device error word 0x%x%s%s", err, (err & kErrWaitTimeout) ? " wait-timeout" : "",
+           (err & kErrPlanShort) ? " plan-short" : "");
+  set_last_error("rswa_decode_noalloc: ", msg);
+  return RSWA_ERR_DEVICE;
 }

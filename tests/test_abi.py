@@ -99,7 +99,21 @@ def test_null_handle_is_an_argument_error(lib):
     assert lib.rswa_reset(None) == _native.ERR_ARG
     assert lib.rswa_check(None) == _native.ERR_ARG
     assert lib.rswa_cache_len(None, None) == _native.ERR_ARG
+    assert lib.rswa_load_reference_chunk(None, None, None, 1, None) == _native.ERR_ARG
     lib.rswa_destroy(None)  # no-op
+
+
+def test_layers_call_rejects_bad_arguments_before_device(lib):
+    P = C.c_void_p * 2
+    buf = C.create_string_buffer(256)
+    p = (C.cast(buf, C.c_void_p).value + 15) // 16 * 16
+    ptrs = P(p, p)
+    f = lib.rswa_append_decode_layers
+    assert f(None, 2, ptrs, ptrs, ptrs, ptrs, 0.0) == _native.ERR_ARG
+    assert f(P(None, None), 2, ptrs, ptrs, ptrs, ptrs, 0.0) == _native.ERR_ARG   # null handles
+    assert f(P(None, None), 0, ptrs, ptrs, ptrs, ptrs, 0.0) == _native.ERR_ARG   # R < 1
+    assert f(P(None, None), 2, ptrs, ptrs, ptrs, ptrs, float("inf")) == _native.ERR_ARG
+    assert f(P(None, None), 2, None, ptrs, ptrs, ptrs, 0.0) == _native.ERR_ARG
 
 
 def test_masked_forward_rejects_bad_arguments_before_device(lib):
