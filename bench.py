@@ -3,14 +3,15 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-Workload (default): single-document bf16 decode -- batch 1, 10 heads, head
-dim 128, L_m = 2592 reference rows (10 pages x 256 vision tokens + 32 prompt
-tokens), window n = 128, outputs continuing past T = 6144.  One "step" decodes
-one output token: the fused append+decode kernel runs once for each of R
-layer caches (R distinct caches, as in an R-layer decoder), so the bytes one
-step touches exceed twice the L2 size and nothing is served from L2 between
-steps.  The timed steps start in the steady state (T > n), where the R-SWA
-cost per step is constant and maximal.
+Headline workload: single-document bf16 decode -- batch 1, 10 heads, head dim
+128, L_m = 2592 reference rows (10 pages x 256 vision tokens + 32 prompt
+tokens), window n = 128, the timed steps ending at output T = 6144.  One
+"step" decodes one output token: the fused append+decode kernel runs once for
+each of R layer caches (R distinct caches, as in an R-layer decoder), so the
+bytes one step touches exceed twice the L2 size and nothing is served from
+L2 between steps.  Every cache is loaded straight at the step the run starts
+from (rswa_load_packed), in the steady state T > n where the R-SWA cost per
+step is constant; exactly K steps are timed.
 
 value     : tokens/s through one attention layer = B * R * K / device time.
 e2e       : the same through the public binding with HOST buffers: every step
@@ -19,10 +20,17 @@ e2e       : the same through the public binding with HOST buffers: every step
 roofline  : algorithmic bytes per launch (2 * rows * d * 2 bytes of K and V
             plus q, o, new k, v) / average launch time, against the measured
             HBM copy bandwidth.
+configs   : (1 GPU) the same measurement for the ragged batch (64 sequences
+            of 2-50 pages, ending at T = 6144) and the long-horizon run
+            (batch 8, 50 pages, ending at T = 100000).
+prefill   : the 32K teacher-forced masked prefill on the tensor cores.
+vs_output_length: per-step latency against T for the R-SWA cache and for the
+            same kernel over the full cache, single document to T = 6144 and
+            long horizon to T = 100000 (the full cache further, to 1e6).
 
 N > 1 GPUs (one process per GPU under torchrun) run independent replicas of
-the workload (R-SWA shards by sequence with no exchange): value is the sum
-of all ranks' tokens over the slowest rank's time.
+the headline workload (R-SWA shards by sequence with no exchange): value is
+the sum of all ranks' tokens over the slowest rank's time.
 """
 
 from __future__ import annotations
@@ -47,12 +55,12 @@ FALLBACK_HBM_GBS = 6650.0
 WORKLOADS = {
     "single_doc": dict(B=1, H=10, d=128, pages=[10], prompt=32, n=128, T=6144, dtype="bf16",
                        desc="single-document bf16 decode: batch 1, 10 heads, d=128, L_m=2592 "
-                            "(10 pages x 256 + 32), n=128, T=6144"),
+                            "(10 pages x 256 + 32), n=128, outputs to T=6144"),
     "ragged": dict(B=64, H=10, d=128, pages=None, prompt=32, n=128, T=6144, dtype="bf16",
                    desc="ragged batched bf16 decode: 64 sequences, pages~U[2,50], "
-                        "L_m=256*pages+32, 10 heads, d=128, n=128, T=6144"),
+                        "L_m=256*pages+32, 10 heads, d=128, n=128, outputs to T=6144"),
     "long": dict(B=8, H=10, d=128, pages=[50] * 8, prompt=32, n=128, T=100000, dtype="bf16",
-                 desc="long-horizon bf16 decode: batch 8, L_m=12832, 10 heads, d=128, n=128, T=100000"),
+                 desc="long-horizon bf16 decode: batch 8, L_m=12832, 10 heads, d=128, n=128, outputs to T=100000"),
 }
 
 
@@ -103,6 +111,11 @@ def measured_tensor_peak():
 
 
 CURVE_T = (1, 32, 64, 128, 256, 512, 1024, 2048, 4096, 6144)
+# long-horizon workload: out to T = 100000, and the full cache further, to
+# 1,000,000 outputs (a 41.5 GB cache for batch 8; loading it needs as much
+# again for its source, so that is as far as half of HBM takes it)
+CURVE_T_LONG = (1, 128, 1024, 8192, 32768, 65536, 100000)
+CURVE_T_LONG_FULL = CURVE_T_LONG + (250000, 500000, 1000000)
 
 
 def cache_rows(lens, n, T, full):
@@ -118,56 +131,74 @@ def curve_cache_ratio(lens, n, Ts):
     return [round(cache_rows(lens, n, T, False) / cache_rows(lens, n, T, True), 6) for T in Ts]
 
 
-def run_curve(w, lens, samples: int = 8):
+def packed_source(B, S, H, d, dtype, seed, block_rows=65536):
+    """A packed [B, S, H, d] tensor of N(0,1) values for loading a cache
+    state with load_packed.  Rows beyond ``block_rows`` repeat the first
+    block (the values do not matter for timing; this keeps the set-up fast
+    for the multi-GB full caches)."""
+    import torch
+    from reference_sliding_window_b200 import synth
+    dev = torch.device("cuda", torch.cuda.current_device())
+    out = torch.empty((B, S, H, d), dtype=synth.torch_dtype(dtype), device=dev)
+    blk = min(S, block_rows)
+    out[:, :blk] = synth.normal((B, blk, H, d), seed, dtype, "cuda")
+    for r0 in range(blk, S, blk):
+        r1 = min(S, r0 + blk)
+        out[:, r0:r1] = out[:, :r1 - r0]
+    return out
+
+
+def run_curve(w, lens, Ts, full_Ts=None, samples: int = 8):
     """Per-step decode latency against the output length T, for the R-SWA
     cache and for the same kernel over the full cache (every output kept):
-    the constant-cost curve against the growing one.  Each sample is one
+    the constant-cost curve against the growing one.  Each cache state is
+    loaded straight at T - 1 outputs (rswa_load_packed); each sample is one
     fused append+decode launch, timed alone with CUDA events after an L2
-    flush; the median of `samples` consecutive steps is reported at each T."""
+    flush; the median of `samples` consecutive steps (outputs T .. T +
+    samples - 1) is reported at each T."""
     import torch
     from reference_sliding_window_b200 import MODE_FULL, MODE_RSWA, RSWA, synth
     dev = torch.device("cuda", torch.cuda.current_device())
     B, H, d, n = w["B"], w["H"], w["d"], w["n"]
     dt = synth.torch_dtype(w["dtype"])
     s = 2 if w["dtype"] == "bf16" else 4
+    full_Ts = tuple(full_Ts or Ts)
     L_m_cap = max(lens)
-    T_top = CURVE_T[-1] + samples + 1
     flush = torch.empty(2 * torch.cuda.get_device_properties(dev).L2_cache_size, dtype=torch.uint8, device=dev)
     pool = synth.normal((16, 3, B, H, d), 4000, w["dtype"], "cuda")
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    out = {"T": list(CURVE_T), "samples": samples, "timing": "isolated launches after an L2 flush, median",
-           "cache_ratio": curve_cache_ratio(lens, n, CURVE_T)}
-    for name, mode in (("rswa", MODE_RSWA), ("full", MODE_FULL)):
+    out = {"timing": "isolated launches after an L2 flush, median of consecutive steps", "samples": samples,
+           "state": "each point's cache loaded at T-1 outputs with rswa_load_packed"}
+    for name, mode, pts in (("rswa", MODE_RSWA, tuple(Ts)), ("full", MODE_FULL, full_Ts)):
+        T_top = max(pts) + samples
+        src_K = packed_source(B, L_m_cap + T_top, H, d, w["dtype"], 4100)
+        src_V = packed_source(B, L_m_cap + T_top, H, d, w["dtype"], 4200)
         a = RSWA(L_m_cap, n, H, d, B, dt, mode=mode, T_cap=T_top, device=dev)
-        Kr = synth.normal((B, H, L_m_cap, d), 4100, w["dtype"], "cuda")
-        Vr = synth.normal((B, H, L_m_cap, d), 4200, w["dtype"], "cuda")
-        a.load_reference(Kr, Vr, lens)
-        del Kr, Vr
         o = torch.empty((B, H, d), dtype=dt, device=dev)
-        T, us, gbs = 0, [], []
-        for Tc in CURVE_T:
-            while T < Tc - 1:  # the next launch appends output Tc
-                x = pool[T % 16]
-                a.append_decode(x[0], x[1], x[2], out=o)
-                T += 1
+        us, gbs = [], []
+        for Tc in pts:
+            a.load_packed(src_K, src_V, lens, Tc - 1)
             ts = []
-            for _ in range(samples):
-                x = pool[T % 16]
+            for i in range(samples):
+                x = pool[i % 16]
                 flush.zero_()
                 e0.record()
                 a.append_decode(x[0], x[1], x[2], out=o)
                 e1.record()
                 e1.synchronize()
                 ts.append(e0.elapsed_time(e1) * 1e3)
-                T += 1
             t_us = statistics.median(ts)
             rows = cache_rows(lens, n, Tc, mode == MODE_FULL)
             us.append(round(t_us, 2))
             gbs.append(round(H * (2 * rows * d * s + 4 * B * d * s) / t_us / 1e3, 1))
         a.check()
+        out[f"{name}_T"] = list(pts)
         out[f"{name}_us"] = us
         out[f"{name}_gbs"] = gbs
-        del a
+        out[f"{name}_cache_gb"] = round(2 * H * d * s * cache_rows(lens, n, max(pts), mode == MODE_FULL) / 1e9, 3)
+        del a, src_K, src_V
+        torch.cuda.empty_cache()
+    out["cache_ratio"] = curve_cache_ratio(lens, n, Ts)
     return out
 
 
@@ -401,10 +432,32 @@ def bytes_per_launch(w, lens):
     return sum(H * (2 * (L + n) * d * s + 4 * d * s) for L in lens)
 
 
-def run_ours(args, w, lens):
+GRAPH_STEPS = 16  # decode steps per captured CUDA graph
+
+
+def step_plan(T_target: int, n: int, steps: int, warmup: int):
+    """Where the decode run starts: the cache is loaded at T0 outputs, then
+    `warmup` eager steps and one graph replay of GRAPH_STEPS warm-up steps
+    run, then exactly `steps` timed steps, ending at output T_target when
+    that leaves the ring full (T0 >= n) at the start; otherwise T0 = n and
+    the run ends past T_target.  -> (T0, first timed output, last)."""
+    T0 = max(n, T_target - warmup - GRAPH_STEPS - steps)
+    first = T0 + warmup + GRAPH_STEPS + 1
+    return T0, first, first + steps - 1
+
+
+def run_decode(args, name, w, lens, T_target, steps, warmup, e2e_steps):
+    """Times `steps` decode steps of workload w.  One step runs the fused
+    append+decode once for each of R layer caches (R distinct caches, as in
+    an R-layer decoder, with R * bytes per launch >= 2 x L2 so nothing is
+    served from L2 between steps).  Every cache starts at T0 outputs
+    (rswa_load_packed from a packed random sequence), in the steady state
+    T > n where the R-SWA cost per step is constant.  The steps run as CUDA
+    graphs of GRAPH_STEPS steps plus one graph for the remainder, so exactly
+    `steps` steps are timed."""
     import torch
     import torch.distributed as dist
-    from reference_sliding_window_b200 import RSWA, synth
+    from reference_sliding_window_b200 import RSWA, append_decode_layers, synth
 
     world, rank, local = dist_env()
     dev = torch.device("cuda", local)
@@ -415,42 +468,48 @@ def run_ours(args, w, lens):
     per_launch = bytes_per_launch(w, lens)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     R = args.layers or max(1, math.ceil(2 * l2 / per_launch))
+    T0, T_first, T_last = step_plan(T_target, n, steps, warmup)
 
-    # R layer caches with their reference segments
     layers = []
     for r in range(R):
         a = RSWA(L_m_cap, n, H, d, B, dt, device=dev)
-        Kr = synth.normal((B, H, L_m_cap, d), replica_seed(1000, r, rank), w["dtype"], "cuda")
-        Vr = synth.normal((B, H, L_m_cap, d), replica_seed(2000, r, rank), w["dtype"], "cuda")
-        a.load_reference(Kr, Vr, lens)
-        del Kr, Vr
+        Kp = packed_source(B, L_m_cap + T0, H, d, w["dtype"], replica_seed(1000, r, rank))
+        Vp = packed_source(B, L_m_cap + T0, H, d, w["dtype"], replica_seed(2000, r, rank))
+        a.load_packed(Kp, Vp, lens, T0)
+        del Kp, Vp
         layers.append(a)
-    P = 16  # distinct per-step inputs, cycled
+    torch.cuda.empty_cache()
+    P = GRAPH_STEPS  # distinct per-step inputs, cycled
     pool = synth.normal((P, R, 3, B, H, d), replica_seed(3000, 0, rank), w["dtype"], "cuda")
     out = torch.empty((R, B, H, d), dtype=dt, device=dev)
+    outs = [out[r] for r in range(R)]
+    # per-step views of the inputs, made once (as a model holds its buffers)
+    views = [([pool[i, r, 0] for r in range(R)], [pool[i, r, 1] for r in range(R)],
+              [pool[i, r, 2] for r in range(R)]) for i in range(P)]
 
     def step(i):
-        x = pool[i % P]
-        for r, a in enumerate(layers):
-            a.append_decode(x[r, 0], x[r, 1], x[r, 2], out=out[r])
+        k, v, q = views[i % P]
+        append_decode_layers(layers, k, v, q, out=outs)
 
+    reps, tail = divmod(steps, P)
     stream = torch.cuda.Stream(device=dev)
     stream.wait_stream(torch.cuda.current_stream(dev))
     with torch.cuda.stream(stream):
-        # fill the ring (steady state) and warm up
-        for i in range(n + args.warmup):
+        for i in range(warmup):
             step(i)
         torch.cuda.synchronize(dev)
-        # capture P steps (R launches each) in one graph
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             for i in range(P):
                 step(i)
-        for _ in range(max(1, args.warmup // P)):
-            g.replay()
+        gt = None
+        if tail:
+            gt = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gt, stream=stream):
+                for i in range(tail):
+                    step(i)
+        g.replay()  # warm-up replay
         torch.cuda.synchronize(dev)
-    reps = max(1, math.ceil(args.steps / P))
-    K = reps * P
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):  # graph replays launch on the current stream
         if dist.is_initialized():
@@ -460,32 +519,34 @@ def run_ours(args, w, lens):
             start.record(stream)
             for _ in range(reps):
                 g.replay()
+            if gt is not None:
+                gt.replay()
             end.record(stream)
             torch.cuda.synchronize(dev)
         if dist.is_initialized():
             dist.barrier()
     elapsed = start.elapsed_time(end) / 1e3
-    launches = K * R
+    launches = steps * R
     for a in layers:
         a.check()
     T_end = layers[0].step_count()[0]
+    assert T_end == T_last, (T_end, T_last)
 
     # ---- e2e: host buffers through the public binding
-    K_e2e = min(K, max(P, args.e2e_steps))
+    K_e2e = max(1, e2e_steps)
     host_in = torch.empty((P, R, 3, B, H, d), dtype=dt, pin_memory=True)
     host_in.copy_(pool.cpu())
     host_out = torch.empty((K_e2e, R, B, H, d), dtype=dt, pin_memory=True)
     dev_in = torch.empty((R, 3, B, H, d), dtype=dt, device=dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     # per-layer views of the staging buffers, made once (as a model holds them)
-    views = [(a, dev_in[r, 0], dev_in[r, 1], dev_in[r, 2], out[r]) for r, a in enumerate(layers)]
+    kv_q = ([dev_in[r, 0] for r in range(R)], [dev_in[r, 1] for r in range(R)], [dev_in[r, 2] for r in range(R)])
     with torch.cuda.stream(stream):
         torch.cuda.synchronize(dev)
         e0.record(stream)
         for i in range(K_e2e):
             dev_in.copy_(host_in[i % P], non_blocking=True)
-            for a, k_r, v_r, q_r, o_r in views:
-                a.append_decode(k_r, v_r, q_r, out=o_r)
+            append_decode_layers(layers, *kv_q, out=outs)
             host_out[i].copy_(out, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize(dev)
@@ -493,23 +554,62 @@ def run_ours(args, w, lens):
     for a in layers:
         a.check()
 
-    el_max, tok_sum = reduce_max_sum(elapsed, float(B * R * K), dev)
+    el_max, tok_sum = reduce_max_sum(elapsed, float(B * R * steps), dev)
     e2e_max, e2e_tok = reduce_max_sum(e2e_s, float(B * R * K_e2e), dev)
     g.reset()
-    return dict(R=R, K=K, elapsed=elapsed, el_max=el_max, tok_sum=tok_sum, launches=launches,
+    if gt is not None:
+        gt.reset()
+    del layers, pool, out, outs, views
+    torch.cuda.empty_cache()
+    s_el = 2 if w["dtype"] == "bf16" else 4
+    return dict(name=name, R=R, K=steps, elapsed=elapsed, el_max=el_max, tok_sum=tok_sum, launches=launches,
                 per_launch=per_launch, clocks=clk.summary(), e2e_max=e2e_max, e2e_tok=e2e_tok,
-                K_e2e=K_e2e, T_end=T_end, l2=l2,
-                h2d=int(R * 3 * B * H * d * (2 if w["dtype"] == "bf16" else 4)),
-                d2h=int(R * B * H * d * (2 if w["dtype"] == "bf16" else 4)))
+                K_e2e=K_e2e, T_range=[T_first, T_last], l2=l2,
+                h2d=int(R * 3 * B * H * d * s_el), d2h=int(R * B * H * d * s_el))
+
+
+def decode_entry(args, w, lens, res, cpu=None):
+    """The JSON fields of one decode workload's measurement."""
+    peak, peak_kind = measured_peaks()
+    avg_launch = res["elapsed"] / res["launches"]
+    achieved = res["per_launch"] / avg_launch / 1e9
+    world = dist_env()[0]
+    config = {"workload": w["desc"] + f"; timed outputs T = {res['T_range'][0]}..{res['T_range'][1]}",
+              "batch": w["B"], "heads": w["H"], "head_dim": w["d"], "n": w["n"],
+              "L_m": lens if len(lens) <= 8 else {"min": min(lens), "max": max(lens),
+                                                  "mean": sum(lens) / len(lens)},
+              "layers_cycled": res["R"],
+              "l2": f"inputs larger than L2: {res['R']} layer cache(s) x {res['per_launch'] / 1e6:.2f} MB "
+                    f"= {res['R'] * res['per_launch'] / 1e6:.0f} MB per step vs L2 {res['l2'] / 1e6:.0f} MB",
+              "T_range": res["T_range"],
+              "unit_def": "one decode token of one attention layer for one sequence",
+              "parallelism": f"replicas x{world}"}
+    return {
+        "value": whole_job_rate(res["tok_sum"], res["el_max"]), "unit": "tokens/s",
+        "steps": res["K"], "ms_per_step": 1e3 * res["el_max"] / res["K"], "config": config,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_kind": f"{peak_kind} HBM copy",
+                     "traffic": recorded_traffic(res["name"]),
+                     "algorithmic_bytes_per_launch": res["per_launch"],
+                     "avg_launch_us": avg_launch * 1e6, "kernel": "rswa::decode_kernel<bf16,128,append>"},
+        "clocks": res["clocks"],
+        "e2e": {"value": whole_job_rate(res["e2e_tok"], res["e2e_max"]), "unit": "tokens/s",
+                "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"], "steps": res["K_e2e"]},
+        "gpu_launches": res["launches"],
+        "cpu_baseline": cpu,
+    }
 
 
 # ------------------------------------------------------------ oracle timing
 
-def oracle_sample(w, lens, budget_s: float, seed: int = 0):
+def oracle_sample(w, lens, budget_s: float, seed: int = 0, max_seqs: int = 4):
     """Times the fp64 CPU oracle on decode steps of this workload: each
-    sampled step recomputes the attention of one token for every sequence
-    and head from the full history (steady state, T = n + a few).  Returns
-    (tokens/s of one layer, threads, description)."""
+    sampled step recomputes the attention of one token for one sequence and
+    every head from the full history (steady state, T = n + a few).  For a
+    batch, up to ``max_seqs`` sequences at evenly spaced quantiles of the
+    reference lengths stand in for the batch and run in turn, so the rate
+    weighs the length mix as the whole batch would.  Returns (tokens/s of
+    one layer, threads, description)."""
     import numpy as np
     import oracle
     try:
@@ -518,23 +618,27 @@ def oracle_sample(w, lens, budget_s: float, seed: int = 0):
     except Exception:
         threads = 1
     rng = np.random.default_rng(seed)
-    B, H, d, n = w["B"], w["H"], w["d"], w["n"]
+    H, d, n = w["H"], w["d"], w["n"]
     T = n + 8
+    srt = sorted(lens)
+    k = min(max_seqs, len(srt))
+    pick = [srt[(2 * i + 1) * len(srt) // (2 * k)] for i in range(k)]
     hist = []
-    for L in lens:
+    for L in pick:
         Kh = rng.standard_normal((L + T, H, d))
         Vh = rng.standard_normal((L + T, H, d))
         hist.append((Kh, Vh))
-    steps, t0 = 0, time.perf_counter()
+    done, t0 = 0, time.perf_counter()
     while True:
         q = rng.standard_normal((H, d))
-        for b, L in enumerate(lens):
-            oracle.decode_step(q, hist[b][0], hist[b][1], L, T, n)
-        steps += 1
+        for i, L in enumerate(pick):
+            oracle.decode_step(q, hist[i][0], hist[i][1], L, T, n)
+        done += len(pick)
         el = time.perf_counter() - t0
-        if el >= budget_s and steps >= 2:
+        if el >= budget_s and done >= 2:
             break
-    return B * steps / el, threads, f"{steps} decode steps x {B} sequences x {H} heads (T={T}), fp64 numpy"
+    who = f"{len(pick)} of {len(lens)} sequences (L_m {pick})" if len(lens) > 1 else f"L_m {pick[0]}"
+    return done / el, threads, f"{done} sequence decode steps x {H} heads (T={T}), {who}, fp64 numpy"
 
 
 def oracle_prefill_sample(w, budget_s: float, seed: int = 0, n_random: int = 256, docs=None):
@@ -582,35 +686,40 @@ def oracle_prefill_sample(w, budget_s: float, seed: int = 0, n_random: int = 256
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=6144)
-    ap.add_argument("--warmup", type=int, default=16)
+    ap.add_argument("--steps", type=int, default=64)
+    ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["prefill", "varlen"], default="single_doc")
+    ap.add_argument("--nested", type=int, default=1,
+                    help="1: with the single-document headline on one GPU, also time the ragged and "
+                         "long-horizon decode workloads")
     ap.add_argument("--prefill-iters", type=int, default=10, help="timed masked-prefill calls (0: skip)")
     ap.add_argument("--curve", type=int, default=1, help="1: add per-step latency vs T, R-SWA and full cache")
     ap.add_argument("--layers", type=int, default=0, help="layer caches cycled (0: 2 x L2 rule)")
-    ap.add_argument("--e2e-steps", type=int, default=256)
+    ap.add_argument("--e2e-steps", type=int, default=64)
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle timing")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.steps < 1:
+        ap.error("--steps must be >= 1")
 
     world, rank, local = dist_env()
     if args.workload in ("prefill", "varlen"):
         return main_prefill(args)
     w = WORKLOADS[args.workload]
     lens = ref_lens_for(w)
-    config = {"workload": w["desc"], "batch": w["B"], "heads": w["H"], "head_dim": w["d"], "n": w["n"],
-              "L_m": lens if len(lens) <= 8 else {"min": min(lens), "max": max(lens), "mean": sum(lens) / len(lens)}}
 
     if args.impl == "reference":
         if rank != 0:
             return 0
         v, threads, sample = oracle_sample(w, lens, args.cpu_budget)
+        config = {"workload": w["desc"], "batch": w["B"], "heads": w["H"], "head_dim": w["d"], "n": w["n"],
+                  "l2": "host CPU"}
         line = {"metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": 1e3 * w["B"] / v, "higher_is_better": True,
+                "warmup": args.warmup, "ms_per_step": 1e3 / v, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "impl": "reference", "config": dict(config, l2="host CPU"),
+                "impl": "reference", "config": config,
                 "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                                  "sample": sample},
                 "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -623,47 +732,38 @@ def main():
         import datetime
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    try:
-        res = run_ours(args, w, lens)
-    finally:
-        pass
-    peak, peak_kind = measured_peaks()
-    avg_launch = res["elapsed"] / res["launches"]
-    achieved = res["per_launch"] / avg_launch / 1e9
-    line = None
+    res = run_decode(args, args.workload, w, lens, w["T"], args.steps, args.warmup, args.e2e_steps)
     if rank == 0:
         cpu = None
         if world == 1:
             v, threads, sample = oracle_sample(w, lens, args.cpu_budget)
             cpu = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample}
-        value = whole_job_rate(res["tok_sum"], res["el_max"])
+        entry = decode_entry(args, w, lens, res, cpu)
+        nested = {}
+        curves = {}
+        if world == 1 and args.nested and args.workload == "single_doc":
+            for name in ("ragged", "long"):
+                wn = WORKLOADS[name]
+                ln = ref_lens_for(wn)
+                rn = run_decode(args, name, wn, ln, wn["T"], args.steps, args.warmup, args.e2e_steps)
+                v, threads, sample = oracle_sample(wn, ln, args.cpu_budget / 3)
+                nested[name] = decode_entry(args, wn, ln, rn, {"value": v, "unit": "tokens/s", "cores": threads,
+                                                               "kind": "oracle", "sample": sample})
         prefill = run_prefill(args.prefill_iters, 3) if (args.prefill_iters > 0 and world == 1) else None
-        curve = run_curve(w, lens) if (args.curve and world == 1 and w["B"] * max(lens) <= 16384) else None
-        line = {
-            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": res["K"],
-            "warmup": args.warmup, "ms_per_step": 1e3 * res["el_max"] / res["K"], "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": w["dtype"], "data": "synthetic",
-            "config": dict(config, layers_cycled=res["R"],
-                           l2=f"inputs larger than L2: {res['R']} layer caches x {res['per_launch'] / 1e6:.2f} MB "
-                              f"= {res['R'] * res['per_launch'] / 1e6:.0f} MB per step vs L2 "
-                              f"{res['l2'] / 1e6:.0f} MB",
-                           T_range=[w["n"] + args.warmup, res["T_end"]],
-                           unit_def="one decode token of one attention layer for one sequence",
-                           parallelism=f"replicas x{world}"),
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "peak_kind": f"{peak_kind} HBM copy",
-                         "traffic": recorded_traffic(args.workload),
-                         "algorithmic_bytes_per_launch": res["per_launch"],
-                         "avg_launch_us": avg_launch * 1e6, "kernel": "rswa::decode_kernel<bf16,128,append>"},
-            "clocks": res["clocks"],
-            "e2e": {"value": whole_job_rate(res["e2e_tok"], res["e2e_max"]), "unit": "tokens/s",
-                    "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"],
-                    "steps": res["K_e2e"]},
-            "gpu_launches": res["launches"],
-            "cpu_baseline": cpu,
-            "prefill": prefill,
-            "vs_output_length": curve,
-        }
+        if args.curve and world == 1 and w["B"] * max(lens) <= 16384:
+            curves[args.workload] = run_curve(w, lens, CURVE_T)
+            if args.nested and args.workload == "single_doc":
+                wl = WORKLOADS["long"]
+                curves["long"] = run_curve(wl, ref_lens_for(wl), CURVE_T_LONG, CURVE_T_LONG_FULL)
+        line = {"metric": METRIC, "value": entry["value"], "unit": "tokens/s", "n_gpus": world,
+                "steps": entry["steps"], "warmup": args.warmup, "ms_per_step": entry["ms_per_step"],
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w["dtype"],
+                "data": "synthetic"}
+        for key in ("config", "roofline", "clocks", "e2e", "gpu_launches", "cpu_baseline"):
+            line[key] = entry[key]
+        line["configs"] = nested or None
+        line["prefill"] = prefill
+        line["vs_output_length"] = curves or None
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

@@ -74,3 +74,23 @@ def test_pack_oracle_baseline_runs_on_a_small_pack():
     v, threads, sample = bench.oracle_prefill_sample(w, budget_s=0.05, n_random=4,
                                                      docs=([0, 120, 121, 300], [40, 1, 0]))
     assert v > 0 and "3 documents" in sample
+
+
+def test_step_plan_times_exactly_the_steps_asked_and_ends_at_the_target():
+    for T_target, n, steps, warmup in [(6144, 128, 20, 5), (100000, 128, 64, 8), (6144, 128, 6144, 8),
+                                       (300, 128, 7, 3)]:
+        T0, first, last = bench.step_plan(T_target, n, steps, warmup)
+        assert T0 >= n  # the ring is full before the first timed step
+        assert last - first + 1 == steps
+        assert first == T0 + warmup + bench.GRAPH_STEPS + 1
+        if T_target - warmup - bench.GRAPH_STEPS - steps >= n:
+            assert last == T_target
+
+
+def test_oracle_sample_weighs_a_ragged_batch_by_quantiles():
+    w = dict(bench.WORKLOADS["ragged"])
+    w.update(H=1, d=16)
+    lens = [100, 200, 300, 400, 500, 600, 700, 800]
+    v, threads, sample = bench.oracle_sample(w, lens, budget_s=0.05, max_seqs=4)
+    assert v > 0 and threads >= 1
+    assert "4 of 8 sequences (L_m [200, 400, 600, 800])" in sample
