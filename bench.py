@@ -283,12 +283,13 @@ def run_varlen(iters: int, warmup: int):
     return {"workload": f"teacher-forced masked prefill over a pack, bf16: {w['L']} rows holding {len(refs)} "
                         f"documents (lengths {[cu[i + 1] - cu[i] for i in range(len(refs))]}, L_m {refs}), "
                         f"10 heads, d=128, n={w['n']}",
-            "ms_per_call": sec * 1e3, "iters": iters, "launches_per_call": len(refs), "tflops": tf,
+            "ms_per_call": sec * 1e3, "iters": iters, "launches_per_call": 1, "tflops": tf,
             "visible_pairs_per_head": pairs,
             "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
-                         "peak_kind": f"{kind} dense bf16 (burst)", "traffic": None,
-                         "algorithmic_flops_per_launch": flops / len(refs),
-                         "kernel": "rswa::tc::masked_tc_kernel (one launch per document)"}}
+                         "peak_kind": f"{kind} dense bf16 (burst)",
+                         "traffic": recorded_traffic("varlen", PREFILL_SOURCES, "prefill_traffic.json"),
+                         "algorithmic_flops_per_launch": flops,
+                         "kernel": "rswa::tc::masked_tc_kernel (the whole pack in one launch)"}}
 
 
 DECODE_SOURCES = ("decode.cu", "common.cuh", "internal.h")
@@ -422,7 +423,7 @@ def ref_lens_for(w, seed=0):
     if w["pages"] is None:
         pages = synth.ragged_page_counts(w["B"], seed=seed)
     else:
-        pages = w["pages"]
+        pages = w["pages"][:w["B"]]
     return [synth.reference_length(p, w["prompt"]) for p in pages]
 
 
@@ -698,6 +699,9 @@ def main():
     ap.add_argument("--layers", type=int, default=0, help="layer caches cycled (0: 2 x L2 rule)")
     ap.add_argument("--e2e-steps", type=int, default=64)
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle timing")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="decode: keep only the first BATCH sequences of the workload (a smaller case of the same "
+                         "kernel, for profiler captures); 0 = all")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -707,8 +711,13 @@ def main():
     world, rank, local = dist_env()
     if args.workload in ("prefill", "varlen"):
         return main_prefill(args)
-    w = WORKLOADS[args.workload]
+    w = dict(WORKLOADS[args.workload])
     lens = ref_lens_for(w)
+    if args.batch:
+        lens = lens[:args.batch]
+        w["B"] = len(lens)
+        w["desc"] += f" (first {len(lens)} sequences)"
+        args.nested = 0
 
     if args.impl == "reference":
         if rank != 0:

@@ -239,8 +239,10 @@ void rswa_destroy(rswa_handle h);
  * L_m = 0 leaves no reference segment: every query sees p-n+1 .. p, the
  * plain sliding window the pages contrast R-SWA with ("vanilla SWA",
  * 核心导读 Fig. 1 and 方法展开 §1), for ablation.
- * BF16 runs on the tcgen05 tensor-core kernel (d = 128), F32 on a SIMT
- * kernel (d = 64 or 128).  Tiles the mask fully hides are skipped.
+ * BF16 with d = 128 runs on the tcgen05 tensor-core kernel.  F32 (d = 64 or
+ * 128) and BF16 with d = 64 run on a CUDA-core kernel (one warp per query
+ * row and head, float32 online softmax), which is exact to float32 rounding
+ * but far slower.  Key tiles (or ranges) the mask fully hides are skipped.
  * ---------------------------------------------------------------------- */
 rswa_status rswa_masked_forward(const void* Q, const void* K, const void* V, void* O,
                                 int L, int L_m, int n, int H, int d, rswa_dtype dtype,
@@ -270,13 +272,35 @@ rswa_status rswa_masked_forward_ex(const void* Q, const void* K, const void* V, 
  *     increasing (every document has at least one row).
  *   ref_lens: HOST int32[n_docs], 0 <= ref_lens[i] <= length of document i.
  *   n_docs >= 1; n, H, d, dtype, scale, flags as in rswa_masked_forward_ex.
- * Every argument is checked before anything is enqueued.  The documents are
- * launched one after another on `stream`, each exactly as
- * rswa_masked_forward_ex on its rows. */
+ * Every argument is checked before anything is enqueued.  BF16 with d = 128
+ * runs the whole pack in one tensor-core launch (one CTA per document, pair
+ * of 128-row query tiles and head, longest first; more than 1024 pairs are
+ * split over several launches); the CUDA-core kernel (F32, or d = 64) is
+ * launched once per document on its rows. */
 rswa_status rswa_masked_forward_varlen(const void* Q, const void* K, const void* V, void* O,
                                        const int32_t* cu_seqlens, const int32_t* ref_lens, int n_docs,
                                        int n, int H, int d, rswa_dtype dtype, float scale, int flags,
                                        void* stream);
+
+/* The teacher-forced form of one sequence that also leaves a handle's cache
+ * ready to decode: O as rswa_masked_forward_ex computes it with the handle's
+ * window (its n; every output for a FULL-mode handle, i.e. plain causal
+ * attention), and the cache rswa_load_reference of rows [0, L_m) followed by
+ * L - L_m appends leaves: the reference rows, "encoded once" here, and the
+ * newest min(n, L - L_m) outputs in their ring slots (FULL mode: all of
+ * them).  The step counter becomes T0 = L - L_m; the next append is output
+ * T0 + 1 (方法展开 §4, Eq.(6) and its queue).
+ *   h: a handle of batch 1 whose dtype and d the tensors share.
+ *   Q, K, V, O: device [L][H][d], as for rswa_masked_forward.
+ *   1 <= L_m <= min(L, L_m_cap); FULL mode needs L - L_m <= T_cap.
+ *   flags: as rswa_masked_forward_ex.
+ * BF16 with d = 128 does both in one tensor-core launch: each CTA copies the
+ * key and value rows of its own query tiles from the tiles it has staged
+ * for the attention into the cache.  Other types run the CUDA-core kernel
+ * and then a copy kernel.  Stream-ordered on the handle's stream; errors are
+ * reported before anything is enqueued. */
+rswa_status rswa_masked_forward_fill(rswa_handle h, const void* Q, const void* K, const void* V, void* O,
+                                     int L, int L_m, float scale, int flags);
 
 /* ------------------------------------------------------------------------
  * Decode without allocation.  The pages have no counterpart to this call;

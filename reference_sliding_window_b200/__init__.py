@@ -170,6 +170,25 @@ class RSWA:
         self._sync_stream()
         check(_native.lib().rswa_load_reference_chunk(self._h, K.data_ptr(), V.data_ptr(), stride, r))
 
+    def prefill(self, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, L_m: int, scale: float = 0.0,
+                out: Optional[torch.Tensor] = None, bidir_prefix: bool = False) -> torch.Tensor:
+        """Teacher-forced attention of one sequence (Q, K, V: [L, H, d]) with
+        this handle's window, that also fills the cache as a reference load of
+        rows [0, L_m) plus L - L_m appends would; decoding continues at output
+        L - L_m + 1.  Batch-1 handles only."""
+        if Q.dim() != 3:
+            raise ValueError("Q must be [L, H, d]")
+        L = Q.shape[0]
+        for name, t in (("Q", Q), ("K", K), ("V", V)):
+            _check_tensor(name, t, (L, self.H, self.d), self.dtype, self.device)
+        O = torch.empty_like(Q) if out is None else out
+        _check_tensor("out", O, (L, self.H, self.d), self.dtype, self.device)
+        self._sync_stream()
+        check(_native.lib().rswa_masked_forward_fill(self._h, Q.data_ptr(), K.data_ptr(), V.data_ptr(), O.data_ptr(),
+                                                      L, int(L_m), float(scale),
+                                                      _native.FLAG_BIDIR_PREFIX if bidir_prefix else 0))
+        return O
+
     def append(self, k: torch.Tensor, v: torch.Tensor) -> None:
         self._vec("k", k)
         self._vec("v", v)

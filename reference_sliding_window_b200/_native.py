@@ -41,6 +41,7 @@ _PROTOS = {
     "rswa_destroy": (None, [_p]),
     "rswa_masked_forward": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _p]),
     "rswa_masked_forward_ex": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _i, _p]),
+    "rswa_masked_forward_fill": (_i, [_p, _p, _p, _p, _p, _i, _i, _f, _i]),
     "rswa_masked_forward_varlen": (_i, [_p, _p, _p, _p, C.POINTER(C.c_int32), C.POINTER(C.c_int32), _i, _i,
                                        _i, _i, _i, _f, _i, _p]),
     "rswa_decode_noalloc": (_i, [_p, _p, _i, C.POINTER(C.c_int32), _p, _p, _i, _i, _i, _i, _f, _p]),

@@ -197,8 +197,6 @@ static void make_plan(rswa_ctx* c) {
     c->n_ctas = Gc;
     return;
   }
-  // At most kMinMergeCap / 2 CTAs, so a slab never has more partials than one
-  // CTA can merge (two slabs at a time) in shared memory.
   const int G = (int)std::min<long long>(std::min(std::min(c->num_sms, c->lay.max_ctas), kMinMergeCap / 2), total);
   c->items.clear();
   c->cta_begin.assign(G + 1, 0);
@@ -807,6 +805,12 @@ extern "C" rswa_status rswa_masked_forward_ex(const void* Q, const void* K, cons
   p.scale_log2 = sc * 1.4426950408889634f;
   p.bidir_prefix = (flags & RSWA_FLAG_BIDIR_PREFIX) ? 1 : 0;
   p.timing = g_timing;
+  const int32_t cu[2] = {0, L}, refs[1] = {L_m};
+  p.cu = cu;
+  p.refs = refs;
+  p.n_docs = 1;
+  p.fill_kc = p.fill_vc = nullptr;
+  p.fill_S_cap = p.fill_n = p.fill_full = 0;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (dtype == RSWA_BF16 && d == 128) {
     RSWA_CUDA(launch_masked_forward_tc(p, s), "masked forward tensor-core kernel");
@@ -842,7 +846,39 @@ extern "C" rswa_status rswa_masked_forward_varlen(const void* Q, const void* K, 
   }
   if ((long long)cu_seqlens[n_docs] * H * d >= (1ll << 31))
     return fail(RSWA_ERR_ARG, "rswa_masked_forward_varlen: tensor too large");
-  // Each document is a contiguous [len][H][d] slice of the pack.
+  if (dtype == RSWA_BF16 && d == 128) {
+    // The tensor-core kernel takes the whole pack in one launch: one CTA per
+    // (document, pair of query tiles, head).
+    int dev = 0, major = 0, minor = 0;
+    RSWA_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+    RSWA_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev), "device attribute");
+    RSWA_CUDA(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev), "device attribute");
+    if (major != 10 || minor != 0)
+      return fail(RSWA_ERR_UNSUPPORTED, "rswa_masked_forward_varlen: device is sm_%d%d; built for sm_100a", major,
+                  minor);
+    MaskedParams p;
+    p.Q = Q;
+    p.K = K;
+    p.V = V;
+    p.O = O;
+    p.L = cu_seqlens[n_docs];
+    p.L_m = 0;
+    p.n = n;
+    p.H = H;
+    p.D = d;
+    const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)d);
+    p.scale_log2 = sc * 1.4426950408889634f;
+    p.bidir_prefix = (flags & RSWA_FLAG_BIDIR_PREFIX) ? 1 : 0;
+    p.timing = g_timing;
+    p.cu = cu_seqlens;
+    p.refs = ref_lens;
+    p.n_docs = n_docs;
+    p.fill_kc = p.fill_vc = nullptr;
+    p.fill_S_cap = p.fill_n = p.fill_full = 0;
+    RSWA_CUDA(launch_masked_forward_tc(p, static_cast<cudaStream_t>(stream)), "masked forward tensor-core kernel");
+    return RSWA_OK;
+  }
+  // CUDA-core kernel: each document is a contiguous [len][H][d] slice of the pack.
   const size_t row_bytes = (size_t)H * d * elem_size(dtype);
   for (int i = 0; i < n_docs; ++i) {
     const size_t off = (size_t)cu_seqlens[i] * row_bytes;
@@ -852,6 +888,87 @@ extern "C" rswa_status rswa_masked_forward_varlen(const void* Q, const void* K, 
                                             scale, flags, stream);
     if (st != RSWA_OK) return st;
   }
+  return RSWA_OK;
+}
+
+extern "C" rswa_status rswa_masked_forward_fill(rswa_handle h, const void* Q, const void* K, const void* V, void* O,
+                                               int L, int L_m, float scale, int flags) {
+  static const char* who = "rswa_masked_forward_fill";
+  if (rswa_status st = check_handle(h)) return st;
+  if (!Q || !K || !V || !O) return fail(RSWA_ERR_ARG, "%s: null tensor", who);
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
+    return fail(RSWA_ERR_ARG, "%s: tensors must be 16-byte aligned", who);
+  if (flags & ~(int)RSWA_FLAG_BIDIR_PREFIX) return fail(RSWA_ERR_ARG, "%s: unknown flags %d", who, flags);
+  if (!(scale == scale) || isinf(scale)) return fail(RSWA_ERR_ARG, "%s: scale not finite", who);
+  if (h->B != 1) return fail(RSWA_ERR_UNSUPPORTED, "%s: the packed form is one sequence; the handle has batch %d", who, h->B);
+  if (L < 1 || L_m < 1 || L_m > L) return fail(RSWA_ERR_ARG, "%s: L=%d L_m=%d (1 <= L_m <= L)", who, L, L_m);
+  if (L_m > h->L_m_cap) return fail(RSWA_ERR_CAPACITY, "%s: L_m=%d above L_m_cap=%d", who, L_m, h->L_m_cap);
+  const int T0 = L - L_m;
+  if (h->mode == RSWA_MODE_FULL && T0 > h->T_cap)
+    return fail(RSWA_ERR_CAPACITY, "%s: %d outputs above T_cap=%d", who, T0, h->T_cap);
+  if ((long long)L * h->H * h->d >= (1ll << 31)) return fail(RSWA_ERR_ARG, "%s: tensor too large", who);
+  if (rswa_status st = use_device(h)) return st;
+  // The attention window: the handle's n, or every output for the full cache.
+  const int n_att = h->mode == RSWA_MODE_RSWA ? h->n : L;
+  h->Lm.assign(1, L_m);
+  h->T_host = T0;
+  h->plan_window = h->mode == RSWA_MODE_RSWA ? h->n : std::min(h->T_cap, std::max(64, (T0 + 63) / 64 * 64));
+  make_plan(h);
+  RSWA_CUDA(cudaMemcpyAsync(h->ws + h->lay.Lm, h->Lm.data(), 4, cudaMemcpyHostToDevice, h->stream),
+            "upload reference lengths");
+  if (rswa_status st = upload_plan(h)) return st;
+  if (h->dtype == RSWA_BF16 && h->d == 128) {
+    // One tensor-core launch computes O and writes the cache rows.
+    int32_t T0_dev = T0;
+    RSWA_CUDA(cudaMemcpyAsync(h->ws + h->lay.T, &T0_dev, 4, cudaMemcpyHostToDevice, h->stream), "set step counter");
+    MaskedParams p;
+    p.Q = Q;
+    p.K = K;
+    p.V = V;
+    p.O = O;
+    p.L = L;
+    p.L_m = L_m;
+    p.n = n_att;
+    p.H = h->H;
+    p.D = h->d;
+    const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)h->d);
+    p.scale_log2 = sc * 1.4426950408889634f;
+    p.bidir_prefix = (flags & RSWA_FLAG_BIDIR_PREFIX) ? 1 : 0;
+    p.timing = g_timing;
+    const int32_t cu[2] = {0, L}, refs[1] = {L_m};
+    p.cu = cu;
+    p.refs = refs;
+    p.n_docs = 1;
+    p.fill_kc = h->kc;
+    p.fill_vc = h->vc;
+    p.fill_S_cap = h->S_cap;
+    p.fill_n = h->mode == RSWA_MODE_RSWA ? h->n : 0;
+    p.fill_full = h->mode == RSWA_MODE_FULL ? 1 : 0;
+    RSWA_CUDA(launch_masked_forward_tc(p, h->stream), "masked forward tensor-core kernel");
+  } else {
+    // CUDA-core attention, then the cache from the same packed rows.
+    if (rswa_status st = rswa_masked_forward_ex(Q, K, V, O, L, L_m, n_att, h->H, h->d, h->dtype, scale, flags,
+                                                h->stream))
+      return st;
+    LoadPackedParams p;
+    p.kc = h->kc;
+    p.vc = h->vc;
+    p.K = K;
+    p.V = V;
+    p.B = 1;
+    p.H = h->H;
+    p.S_cap = h->S_cap;
+    p.row_bytes = h->row_bytes;
+    p.seq_stride = L;
+    p.n = h->n;
+    p.T0 = T0;
+    p.full_mode = h->mode == RSWA_MODE_FULL;
+    p.Lm = ws_i32(h, h->lay.Lm);
+    p.T = ws_i32(h, h->lay.T);
+    const int W = h->mode == RSWA_MODE_RSWA ? std::min(h->n, T0) : T0;
+    RSWA_CUDA(launch_load_packed(p, L_m + W, h->stream), "load_packed kernel");
+  }
+  h->loaded = true;
   return RSWA_OK;
 }
 

@@ -161,6 +161,19 @@ struct MaskedParams {
   float scale_log2;
   int bidir_prefix;             // 1: prefix queries see every reference key
   unsigned long long* timing;  // profiling stamps (RSWA_TIMING builds), may be null
+  // Documents of a pack (tensor-core kernel): document i holds rows
+  // [cu[i], cu[i+1]) with refs[i] reference rows; HOST arrays.  The
+  // single-sequence form is one document {0, L} with L_m reference rows.
+  const int32_t* cu;
+  const int32_t* refs;
+  int n_docs;
+  // Cache fill by the tensor-core kernel (one document): null fill_kc for
+  // none.  Caches [H][fill_S_cap][D]; reference rows at their row; outputs in
+  // a ring of fill_n slots keeping the newest fill_n, or all in order
+  // (fill_full).
+  void* fill_kc;
+  void* fill_vc;
+  int fill_S_cap, fill_n, fill_full;
 };
 // Sets the thread-local message returned by rswa_last_error().
 void set_last_error(const char* prefix, const char* msg);

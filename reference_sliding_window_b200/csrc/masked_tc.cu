@@ -43,16 +43,13 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <algorithm>
 #include <mutex>
+#include <utility>
+#include <vector>
 
 #include "common.cuh"
 #include "internal.h"
-
-// Exponentials per 8 columns of an unmasked tile evaluated on the FMA pipe
-// (the rest use the XU pipe's ex2).
-#ifndef RSWA_EMU_EIGHTHS
-#define RSWA_EMU_EIGHTHS 0  // measured on B200: enabling it slowed the kernel down
-#endif
 
 namespace rswa {
 namespace tc {
@@ -209,20 +206,10 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe, to take part of the exponentials off the XU pipe:
-// n = round(x) with the 1.5*2^23 shifter (Cody-Waite style range reduction),
-// f = x - n in [-1/2, 1/2], 2^f by a cubic, then n is added to the exponent
-// field.  The cubic is the relative least-squares fit of 2^f at Chebyshev
-// nodes computed by fit_exp2.py (relative error <= 7.8e-5, far below the
-// bf16 rounding of P).  For x >= -126 only; callers use it on unmasked tiles.
-__device__ __forceinline__ float exp2_fma(float x) {
-  constexpr float kC0 = 0.99992895f, kC1 = 0.6932762f, kC2 = 0.24260405f, kC3 = 0.055088684f;
-  constexpr float kShift = 12582912.f;  // 1.5 * 2^23
-  x = fmaxf(x, -126.f);
-  const float y = x + kShift;
-  const float f = x - (y - kShift);
-  const float p = fmaf(fmaf(fmaf(kC3, f, kC2), f, kC1), f, kC0);
-  return __int_as_float(__float_as_int(p) + ((__float_as_int(y) - __float_as_int(kShift)) << 23));
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -231,13 +218,30 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// One CTA's work: a pair of query tiles of one document of the pack.
+struct TcWork {
+  int start;  // first pack row of the document
+  int len;    // its rows
+  int ref;    // its reference rows (L_m)
+  int pair;   // the pair of 128-row query tiles, local rows [256*pair, 256*pair + 256)
+};
+constexpr int kMaxWork = 1024;  // table entries per launch (16 KB of kernel parameters)
+
 struct TcParams {
-  CUtensorMap tmQ, tmK, tmV;  // 3-D maps {d, H, L} of bf16, 64x1x128 boxes, 128B swizzle
+  CUtensorMap tmQ, tmK, tmV;  // 3-D maps {d, H, rows} of bf16 over the whole pack, 64x1x128 boxes, 128B swizzle
   __nv_bfloat16* O;
-  int L, L_m, n, H, n_qtiles;
+  int n, H;
   int bidir;                  // 1: prefix queries see every reference key
   float scale_log2;
   unsigned long long* timing;  // RSWA_TIMING builds: per-tile cycle stamps of CTA 0
+  // Optional cache fill (one sequence): K and V rows into [H][S_cap][d]
+  // caches, reference rows at their row, outputs in an n-slot ring that
+  // keeps the newest fill_n of them, or (fill_full) every output in order.
+  __nv_bfloat16* kc;          // null: no fill
+  __nv_bfloat16* vc;
+  int S_cap, fill_n, fill_full;
+  int n_work;
+  TcWork work[kMaxWork];      // heaviest first; CTA c takes entry c / H, head c % H
 };
 
 // RSWA_TIMING builds record clock64 stamps of CTA 0 for its first 32 key
@@ -255,8 +259,8 @@ struct TileRange {
   int A, B0, B1;
 };
 
-__device__ __forceinline__ TileRange tile_range(int q0, int len, int L, int L_m, int n, bool bidir) {
-  const int q_last = min(q0 + len, L) - 1;
+__host__ __device__ __forceinline__ TileRange tile_range(int q0, int len, int L, int L_m, int n, bool bidir) {
+  const int q_last = (q0 + len < L ? q0 + len : L) - 1;
   TileRange r;
   if (q_last < L_m) {  // all prefix rows: causal, or every reference key (bidirectional)
     r.A = bidir ? (L_m + kTile - 1) / kTile : q_last / kTile + 1;
@@ -265,13 +269,16 @@ __device__ __forceinline__ TileRange tile_range(int q0, int len, int L, int L_m,
     return r;
   }
   r.A = (L_m + kTile - 1) / kTile;
-  const int lo = max(L_m, max(q0, L_m) - n + 1);
-  r.B0 = max(r.A, lo / kTile);
+  const int qs = q0 > L_m ? q0 : L_m;
+  const int lo = qs - n + 1 > L_m ? qs - n + 1 : L_m;
+  r.B0 = lo / kTile > r.A ? lo / kTile : r.A;
   r.B1 = q_last / kTile;
   return r;
 }
 
-__device__ __forceinline__ int tile_count(const TileRange& r) { return r.A + max(0, r.B1 - r.B0 + 1); }
+__host__ __device__ __forceinline__ int tile_count(const TileRange& r) {
+  return r.A + (r.B1 - r.B0 + 1 > 0 ? r.B1 - r.B0 + 1 : 0);
+}
 __device__ __forceinline__ int tile_at(const TileRange& r, int j) { return j < r.A ? j : r.B0 + (j - r.A); }
 
 // Barrier slots (8 bytes each).
@@ -286,18 +293,25 @@ enum : int {
 // for a prefix row, and the output window).
 template <bool FULL>
 __device__ __forceinline__ float half_max(const float* s, int col0, int ra, int wb, int we) {
-  float m8[8];  // independent chains: 8 steps deep instead of 64
+  float m8[8];  // independent chains
 #pragma unroll
   for (int k = 0; k < 8; ++k) m8[k] = -INFINITY;
+  if (FULL) {
 #pragma unroll
-  for (int e = 0; e < kHalf; ++e) {
-    const int c = col0 + e;
-    m8[e & 7] = fmaxf(m8[e & 7], (FULL || c < ra || (c >= wb && c <= we)) ? s[e] : -INFINITY);
+    for (int e = 0; e < kHalf; e += 2) m8[(e >> 1) & 7] = max3(m8[(e >> 1) & 7], s[e], s[e + 1]);
+  } else {
+#pragma unroll
+    for (int e = 0; e < kHalf; ++e) {
+      const int c = col0 + e;
+      m8[e & 7] = fmaxf(m8[e & 7], (c < ra || (c >= wb && c <= we)) ? s[e] : -INFINITY);
+    }
   }
-  return fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+  return fmaxf(max3(m8[0], m8[1], m8[2]), max3(m8[3], max3(m8[4], m8[5], m8[6]), m8[7]));
 }
 
-// Exponentials of those 64 columns, packed to bf16 pairs; returns their sum.
+// Exponentials p = 2^(s*sl2 - msub) of those 64 columns, one XU
+// instruction each, packed to bf16 pairs (the PV product's operand); returns
+// their float32 sum.  Masked columns get an argument of -inf, so exactly 0.
 template <bool FULL>
 __device__ __forceinline__ float half_exp(const float* s, int col0, int ra, int wb, int we, float sl2, float msub,
                                           uint32_t* pk) {
@@ -306,13 +320,11 @@ __device__ __forceinline__ float half_exp(const float* s, int col0, int ra, int 
   for (int e = 0; e < kHalf; e += 2) {
     const int c = col0 + e;
     float x0 = fmaf(s[e], sl2, -msub), x1 = fmaf(s[e + 1], sl2, -msub);
-    if (!FULL) {  // masked columns: exponent -inf gives exactly 0
+    if (!FULL) {
       x0 = (c < ra || (c >= wb && c <= we)) ? x0 : -INFINITY;
       x1 = (c + 1 < ra || (c + 1 >= wb && c + 1 <= we)) ? x1 : -INFINITY;
     }
-    // the column pattern choosing the FMA-pipe exponential is a compile-time constant
-    const float p0 = (FULL && (e & 7) < RSWA_EMU_EIGHTHS) ? exp2_fma(x0) : ex2(x0);
-    const float p1 = (FULL && ((e + 1) & 7) < RSWA_EMU_EIGHTHS) ? exp2_fma(x1) : ex2(x1);
+    const float p0 = ex2(x0), p1 = ex2(x1);
     l4[(e >> 1) & 3] += p0 + p1;
     pk[e / 2] = pack_bf16x2(p0, p1);
   }
@@ -331,15 +343,14 @@ __global__ void __launch_bounds__(kThreads, 1) masked_tc_kernel(const __grid_con
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // heaviest pairs first: the pairs holding output rows, then prefix pairs
-  // from the largest down
+  // the host orders the table heaviest first, so the hardware block
+  // scheduler approximates longest-job-first
   const int h = blockIdx.x % p.H;
-  const int rank = blockIdx.x / p.H;
-  const int n_pairs = (p.n_qtiles + kQT - 1) / kQT;
-  const int t_s = p.L_m / (kQT * kTile);  // pairs made only of prefix rows
-  const int pr = rank < n_pairs - t_s ? t_s + rank : t_s - 1 - (rank - (n_pairs - t_s));
-  const int q0 = pr * kQT * kTile;
-  const TileRange tr = tile_range(q0, kQT * kTile, p.L, p.L_m, p.n, p.bidir != 0);
+  const TcWork wk = p.work[blockIdx.x / p.H];
+  const int L = wk.len, L_m = wk.ref;  // the document's geometry, in local rows
+  const int ds = wk.start;             // its first pack row (TMA and output coordinates)
+  const int q0 = wk.pair * kQT * kTile;
+  const TileRange tr = tile_range(q0, kQT * kTile, L, L_m, p.n, p.bidir != 0);
   const int nt = tile_count(tr);
 
   if (threadIdx.x == 0) {
@@ -374,36 +385,93 @@ __global__ void __launch_bounds__(kThreads, 1) masked_tc_kernel(const __grid_con
 
   if (warp == 0 || warp == kVWarp) {
     // ---------------------------------------------------------- producers
-    // warp 0: both Q tiles, then the K ring; warp kVWarp: the V ring
-    if (lane == 0) {
-      const bool is_k = warp == 0;
-      const int ns = is_k ? kKS : kVS;
-      const uint32_t full0 = B(is_k ? kBarKFull : kBarVFull), free0 = B(is_k ? kBarKFree : kBarVFree);
-      const uint32_t dst0 = sbase + (is_k ? kSmK : kSmV);
-      const CUtensorMap* map = is_k ? &p.tmK : &p.tmV;
-      if (is_k) {
-        mbar_arrive_expect_tx(B(kBarQ), kQT * kTileBytes);
-        for (int g = 0; g < kQT; ++g) {
-          tma_load_3d(sbase + kSmQ + g * kTileBytes, &p.tmQ, 0, h, q0 + g * kTile, B(kBarQ));
-          tma_load_3d(sbase + kSmQ + g * kTileBytes + kBoxBytes, &p.tmQ, kBox, h, q0 + g * kTile, B(kBarQ));
+    // warp 0: both Q tiles, then the K ring; warp kVWarp: the V ring.  Lane 0
+    // issues the copies; with a cache to fill, the whole warp also copies
+    // this CTA's own key rows (its query rows, whose tiles it loads anyway)
+    // from each staged tile into the cache before the stage is reused.
+    const bool is_k = warp == 0;
+    const int ns = is_k ? kKS : kVS;
+    const uint32_t full0 = B(is_k ? kBarKFull : kBarVFull), free0 = B(is_k ? kBarKFree : kBarVFree);
+    const uint32_t dst0 = sbase + (is_k ? kSmK : kSmV);
+    const CUtensorMap* map = is_k ? &p.tmK : &p.tmV;
+    const bool fill = p.kc != nullptr;
+    const int own_lo = q0 / kTile, own_hi = (min(q0 + kQT * kTile, L) - 1) / kTile;  // this CTA's query tiles
+    // Rows of tile j (staged in stage s) that belong to this CTA's query rows
+    // and to the cache: the reference rows, and the outputs the cache keeps
+    // (the newest fill_n in an n-slot ring, or all of them in FULL mode).
+    auto fill_tile = [&](int j, int s) {
+      const int kt = tile_at(tr, j);
+      if (kt < own_lo || kt > own_hi) return;
+      const uint8_t* base = smem + (is_k ? kSmK : kSmV) + s * kTileBytes;
+      __nv_bfloat16* cache = is_k ? p.kc : p.vc;
+#pragma unroll 4
+      for (int i = 0; i < kTile / 2; ++i) {
+        const int r = 2 * i + (lane >> 4);  // tile row
+        const int c = lane & 15;            // 16-byte chunk of the 256-byte row
+        const int pos = kt * kTile + r;     // local row
+        int crow = -1;
+        if (pos < L) {
+          if (pos < L_m || p.fill_full) crow = pos;
+          else if (pos >= L - p.fill_n) crow = L_m + (pos - L_m) % p.fill_n;
+        }
+        if (crow >= 0) {
+          const uint4 v = *reinterpret_cast<const uint4*>(base + (c >> 3) * kBoxBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+          *reinterpret_cast<uint4*>(cache + ((size_t)h * p.S_cap + crow) * kD + c * 8) = v;
         }
       }
-      int issued = 0;
+    };
+    // A stage's tile is read here only after its full phase completed (the
+    // TMA writes are then visible to this warp).
+    auto wait_full = [&](int j) -> bool {
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait_bounded(full0 + 8u * (j % ns), (j / ns) & 1);
+      return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    };
+    if (lane == 0 && is_k) {
+      mbar_arrive_expect_tx(B(kBarQ), kQT * kTileBytes);
+      for (int g = 0; g < kQT; ++g) {
+        tma_load_3d(sbase + kSmQ + g * kTileBytes, &p.tmQ, 0, h, ds + q0 + g * kTile, B(kBarQ));
+        tma_load_3d(sbase + kSmQ + g * kTileBytes + kBoxBytes, &p.tmQ, kBox, h, ds + q0 + g * kTile, B(kBarQ));
+      }
+    }
+    int issued = 0;
+    if (fill || lane == 0) {
       for (int j = 0; j < nt; ++j) {
         const int s = j % ns;
-        if (*s_abort || !mbar_wait_bounded(free0 + 8u * s, ((j / ns) & 1) ^ 1)) {
-          *s_abort = 1;
+        int ok = 1;
+        if (lane == 0) ok = !*s_abort && mbar_wait_bounded(free0 + 8u * s, ((j / ns) & 1) ^ 1);
+        if (fill) ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) {
+          if (lane == 0) *s_abort = 1;
           break;
         }
-        const int k0 = tile_at(tr, j) * kTile;
-        mbar_arrive_expect_tx(full0 + 8u * s, kTileBytes);
-        tma_load_3d(dst0 + s * kTileBytes, map, 0, h, k0, full0 + 8u * s);
-        tma_load_3d(dst0 + s * kTileBytes + kBoxBytes, map, kBox, h, k0, full0 + 8u * s);
+        if (fill && j >= ns) {
+          if (!wait_full(j - ns)) break;
+          fill_tile(j - ns, s);
+          __syncwarp();  // every lane's reads of the stage before it is loaded again
+        }
+        if (lane == 0) {
+          // rows past the document's end (the next document's, or zero fill
+          // past the pack) are never visible: keys by causality, queries are
+          // not stored
+          const int k0 = ds + tile_at(tr, j) * kTile;
+          mbar_arrive_expect_tx(full0 + 8u * s, kTileBytes);
+          tma_load_3d(dst0 + s * kTileBytes, map, 0, h, k0, full0 + 8u * s);
+          tma_load_3d(dst0 + s * kTileBytes + kBoxBytes, map, kBox, h, k0, full0 + 8u * s);
+        }
         issued = j + 1;
       }
+      // the last staged tiles: fill from them once they have landed
+      if (fill)
+        for (int j = max(0, issued - ns); j < issued; ++j)
+          if (wait_full(j)) fill_tile(j, j % ns);
       // drain: every issued copy has landed before the CTA may exit
-      if (is_k) mbar_wait_bounded(B(kBarQ), 0);
-      for (int j = max(0, issued - ns); j < issued; ++j) mbar_wait_bounded(full0 + 8u * (j % ns), (j / ns) & 1);
+      if (lane == 0) {
+        if (is_k) mbar_wait_bounded(B(kBarQ), 0);
+        for (int j = max(0, issued - ns); j < issued; ++j) mbar_wait_bounded(full0 + 8u * (j % ns), (j / ns) & 1);
+      }
+      // decode kernels may copy reference rows before their dependency wait
+      if (fill) __threadfence();
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
@@ -482,14 +550,14 @@ __global__ void __launch_bounds__(kThreads, 1) masked_tc_kernel(const __grid_con
       if (stamp) TC_CYC(j, 1);
       tc_fence_after();
       const int k0 = tile_at(tr, j) * kTile;
-      const bool full = (k0 + kTile - 1 < p.L_m) && (p.bidir || q0g >= p.L_m || k0 + kTile - 1 <= q0g);
+      const bool full = (k0 + kTile - 1 < L_m) && (p.bidir || q0g >= L_m || k0 + kTile - 1 <= q0g);
       int ra = kTile, wb = 1, we = 0;
       if (!full) {
-        if (i < p.L_m) {
-          ra = (p.bidir ? p.L_m : i + 1) - k0;
+        if (i < L_m) {
+          ra = (p.bidir ? L_m : i + 1) - k0;
         } else {
-          ra = p.L_m - k0;
-          wb = max(p.L_m, i - p.n + 1) - k0;
+          ra = L_m - k0;
+          wb = max(L_m, i - p.n + 1) - k0;
           we = i - k0;
         }
       }
@@ -549,13 +617,13 @@ __global__ void __launch_bounds__(kThreads, 1) masked_tc_kernel(const __grid_con
     tc_fence_after();
     if (!ok) *s_abort = 1;
     const float inv = (ok && !*s_abort) ? 1.f / l_sum : __int_as_float(0x7fc00000);
-    __nv_bfloat16* orow = p.O + ((size_t)i * p.H + h) * kD;
+    __nv_bfloat16* orow = p.O + ((size_t)(ds + i) * p.H + h) * kD;
 #pragma unroll 1
     for (int c = 0; c < kD; c += 32) {
       float o[32];
       tmem_ld32(lane_base + colO + c, o);
       tmem_wait_ld();
-      if (i < p.L) {
+      if (i < L) {
 #pragma unroll
         for (int e = 0; e < 32; e += 8) {
           uint4 w;
@@ -608,32 +676,56 @@ static bool make_map(CUtensorMap* m, const void* base, int L, int H) {
 
 }  // namespace tc
 
+// Launches the kernel over the documents of the pack (one document for the
+// single-sequence form): every (document, pair of query tiles, head) is one
+// CTA.  Entries are ordered by their number of key tiles, heaviest first;
+// a pack with more than kMaxWork pairs is split over several launches.
 cudaError_t launch_masked_forward_tc(const MaskedParams& mp, cudaStream_t stream) {
   using namespace tc;
-  TcParams p;
-  if (!make_map(&p.tmQ, mp.Q, mp.L, mp.H) || !make_map(&p.tmK, mp.K, mp.L, mp.H) ||
-      !make_map(&p.tmV, mp.V, mp.L, mp.H))
+  static TcParams p;  // 16 KB: built in static storage, copied by the launch
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  const int rows = mp.cu[mp.n_docs];
+  if (!make_map(&p.tmQ, mp.Q, rows, mp.H) || !make_map(&p.tmK, mp.K, rows, mp.H) ||
+      !make_map(&p.tmV, mp.V, rows, mp.H))
     return cudaErrorInvalidValue;
   p.O = static_cast<__nv_bfloat16*>(mp.O);
-  p.L = mp.L;
-  p.L_m = mp.L_m;
   p.n = mp.n;
   p.H = mp.H;
-  p.n_qtiles = (mp.L + kTile - 1) / kTile;
   p.scale_log2 = mp.scale_log2;
   p.bidir = mp.bidir_prefix;
   p.timing = mp.timing;
-  static bool configured[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(masked_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmBytes);
-    if (e != cudaSuccess) return e;
-    configured[dev] = true;
+  p.kc = static_cast<__nv_bfloat16*>(mp.fill_kc);
+  p.vc = static_cast<__nv_bfloat16*>(mp.fill_vc);
+  p.S_cap = mp.fill_S_cap;
+  p.fill_n = mp.fill_n;
+  p.fill_full = mp.fill_full;
+  static PerContextOnce attr_once;
+  cudaError_t e = attr_once.run(
+      [] { return cudaFuncSetAttribute(masked_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmBytes); });
+  if (e != cudaSuccess) return e;
+  std::vector<std::pair<int, TcWork>> work;  // (key tiles, entry)
+  auto flush = [&]() -> cudaError_t {
+    if (work.empty()) return cudaSuccess;
+    std::stable_sort(work.begin(), work.end(),
+                     [](const std::pair<int, TcWork>& a, const std::pair<int, TcWork>& b) { return a.first > b.first; });
+    p.n_work = (int)work.size();
+    for (size_t i = 0; i < work.size(); ++i) p.work[i] = work[i].second;
+    masked_tc_kernel<<<p.n_work * p.H, kThreads, kSmBytes, stream>>>(p);
+    work.clear();
+    return cudaGetLastError();
+  };
+  for (int d = 0; d < mp.n_docs; ++d) {
+    const int len = mp.cu[d + 1] - mp.cu[d];
+    const int n_pairs = (len + kQT * kTile - 1) / (kQT * kTile);
+    for (int pr = 0; pr < n_pairs; ++pr) {
+      const TileRange tr = tile_range(pr * kQT * kTile, kQT * kTile, len, mp.refs[d], mp.n, mp.bidir_prefix != 0);
+      work.push_back({tile_count(tr), TcWork{mp.cu[d], len, mp.refs[d], pr}});
+      if ((int)work.size() == kMaxWork)
+        if ((e = flush()) != cudaSuccess) return e;
+    }
   }
-  masked_tc_kernel<<<(p.n_qtiles + kQT - 1) / kQT * p.H, kThreads, kSmBytes, stream>>>(p);
-  return cudaGetLastError();
+  return flush();
 }
 
 }  // namespace rswa

@@ -100,6 +100,7 @@ def test_null_handle_is_an_argument_error(lib):
     assert lib.rswa_check(None) == _native.ERR_ARG
     assert lib.rswa_cache_len(None, None) == _native.ERR_ARG
     assert lib.rswa_load_reference_chunk(None, None, None, 1, None) == _native.ERR_ARG
+    assert lib.rswa_masked_forward_fill(None, None, None, None, None, 8, 4, 0.0, 0) == _native.ERR_ARG
     lib.rswa_destroy(None)  # no-op
 
 

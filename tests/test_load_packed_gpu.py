@@ -10,7 +10,7 @@ import pytest
 import torch
 
 import oracle
-from reference_sliding_window_b200 import MODE_FULL, RSWA, RSWAError, masked_forward, synth
+from reference_sliding_window_b200 import MODE_FULL, MODE_RSWA, RSWA, RSWAError, masked_forward, synth
 from tests.gpu_util import assert_close, compare_steps, make_attn, run_steps
 
 pytestmark = pytest.mark.gpu
@@ -136,3 +136,62 @@ def test_load_packed_rejects_bad_sizes():
         a.load_packed(Kp[:1], Vp[:1], case.ref_lens, 0)
     with pytest.raises(RSWAError, match="STATE"):
         a.decode(torch.zeros(2, 2, 64, device="cuda"))  # nothing loaded yet
+
+
+@pytest.mark.parametrize("dtype,d,L,L_m,n,mode,bidir", [
+    ("bf16", 128, 1000, 300, 128, MODE_RSWA, False),   # the ring's rows span two key tiles
+    ("bf16", 128, 700, 256, 64, MODE_RSWA, False),     # L_m on a tile boundary
+    ("bf16", 128, 2000, 513, 200, MODE_RSWA, True),    # ring wider than a tile; bidirectional prefix
+    ("bf16", 128, 300, 300, 16, MODE_RSWA, False),     # no outputs yet: reference only
+    ("bf16", 128, 400, 399, 16, MODE_RSWA, False),     # one output
+    ("bf16", 128, 700, 300, 16, MODE_FULL, False),     # full cache: every output kept
+    ("f32", 64, 500, 200, 32, MODE_RSWA, False),       # CUDA-core path: attention, then a copy
+])
+def test_prefill_fill_leaves_the_cache_of_a_load_plus_appends(dtype, d, L, L_m, n, mode, bidir, plan):
+    """rswa_masked_forward_fill: O bit for bit the plain masked forward's,
+    the cache bit for bit rswa_load_packed's (which tests above pin to a
+    reference load plus appends), and decoding continues in agreement with
+    the oracle, on spiked queries."""
+    H, T0, extra = 2, L - L_m, 9
+    Q, K, V = synth.prefill_case(L + extra, H, d, dtype, seed=L + n + 61)
+    full = mode == MODE_FULL
+    T_cap = T0 + extra if full else 0
+    n_att = L if full else n
+    Qc, Kc, Vc = Q[:L].cuda(), K[:L].cuda(), V[:L].cuda()
+    a = RSWA(L_m, n, H, d, 1, synth.torch_dtype(dtype), mode=mode, T_cap=T_cap)
+    O = a.prefill(Qc, Kc, Vc, L_m=L_m, bidir_prefix=bidir)
+    O_ref = masked_forward(Qc, Kc, Vc, L_m=L_m, n=n_att, bidir_prefix=bidir)
+    ref = RSWA(L_m, n, H, d, 1, synth.torch_dtype(dtype), mode=mode, T_cap=T_cap)
+    ref.load_packed(Kc, Vc, [L_m], T0)
+    torch.cuda.synchronize()
+    assert torch.equal(O, O_ref)
+    assert a.step_count() == [T0]
+    assert np.array_equal(a.cache_positions(0), ref.cache_positions(0))
+    occ = a.cache_len()[0]
+    assert torch.equal(a.k_cache[0, :, :occ], ref.k_cache[0, :, :occ])
+    assert torch.equal(a.v_cache[0, :, :occ], ref.v_cache[0, :, :occ])
+    # decode outputs T0+1 .. T0+extra: packed rows L .. L+extra-1 are their tokens
+    rows = list(range(L, L + extra))
+    Qs = synth.spike_packed_queries(Q, K, [(r, r - (n if not full else 1) + 1) for r in rows])
+    Kd, Vd, Qd = K.double().numpy(), V.double().numpy(), Qs.double().numpy()
+    want = oracle.masked_forward_rows(Qd, Kd, Vd, L_m, n_att, rows, bidir_prefix=bidir)
+    for i, r in enumerate(rows):
+        o = a.append_decode(K[r].unsqueeze(0).cuda(), V[r].unsqueeze(0).cuda(), Qs[r].unsqueeze(0).cuda())
+        torch.cuda.synchronize()
+        assert_close(o[0], want[i], dtype, f"decode after fill, row {r}")
+    a.check()
+
+
+def test_prefill_fill_rejects_bad_arguments():
+    a = RSWA(100, 8, 2, 128, 2, torch.bfloat16)
+    Q = torch.zeros(120, 2, 128, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(RSWAError, match="UNSUPPORTED"):  # batch 2
+        a.prefill(Q, Q, Q, L_m=100)
+    b = RSWA(100, 8, 2, 128, 1, torch.bfloat16)
+    with pytest.raises(RSWAError, match="CAPACITY"):
+        b.prefill(Q, Q, Q, L_m=101)
+    with pytest.raises(RSWAError, match="ARG"):
+        b.prefill(Q, Q, Q, L_m=0)
+    c = RSWA(100, 8, 2, 128, 1, torch.bfloat16, mode=MODE_FULL, T_cap=10)
+    with pytest.raises(RSWAError, match="CAPACITY"):
+        c.prefill(Q, Q, Q, L_m=100)  # 20 outputs > T_cap
