@@ -47,9 +47,11 @@
 //   slab leave a partial (m, l, o).  Span plan: one release fence and a
 //   relaxed ticket per split item; the CTA holding a slab's last ticket
 //   acquires and merges the slab's partials with the log-sum-exp rule (one
-//   round of independent loads).  Cluster plan: each CTA stores its partial
-//   into the leader CTA's shared memory and arrives on the leader's
-//   mbarrier (release, cluster scope); the leader waits and merges.
+//   round of independent loads).  Cluster plan: each CTA writes its partial
+//   into its own shared memory and one thread sends it to the leader CTA's
+//   shared memory with a bulk copy that completes bytes on the leader's
+//   mbarrier (no release fence or arrival round trip); the leader, whose
+//   barrier expects the other CTAs' bytes, waits and merges.
 // * APPEND: the consumer that meets the slot row substitutes the new k/v
 //   (the staged copy of that row may predate the write) and stores them into
 //   the slot.  Each CTA reads the step counter T once and then takes a
@@ -175,20 +177,14 @@ __device__ __forceinline__ uint32_t cluster_map(uint32_t addr, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
   return r;
 }
-__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
-  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_remote_release(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
 // Every thread of every CTA of the cluster (all threads must execute it).
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 // Bounded wait on a local mbarrier phase with cluster-scope acquire (the
-// arrivals came from other CTAs of the cluster).  Its limit is four times
-// the others': a CTA whose own waits timed out still arrives, about one
-// limit late, and the leader must outlive every store into its shared
+// bytes came from other CTAs of the cluster).  Its limit is four times the
+// others': a CTA whose own waits timed out still sends its partial, about
+// one limit late, and the leader must outlive every copy into its shared
 // memory.
 __device__ __forceinline__ bool mbar_wait_cluster_bounded(uint32_t bar, uint32_t parity) {
   const long long t0 = clock64();
@@ -206,6 +202,13 @@ __device__ __forceinline__ bool mbar_wait_cluster_bounded(uint32_t bar, uint32_t
   }
 }
 
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void bulk_s2cluster(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(dst), "r"(src), "r"(bytes), "r"(bar) : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void griddep_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -300,7 +303,7 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
       mbar_init(smem_u32(&empty_bar[s]), 32 * Tr::kSplit);  // every lane of the owning group
     }
     *s_abort = 0;
-    if (p.cluster_merge) mbar_init(cl_bar, kDecodeCluster);  // one arrival per CTA of the cluster
+    if (p.cluster_merge) mbar_init(cl_bar, 1);  // the leader's own arrival; the others complete bytes
     fence_barrier_init();
   }
   // The plan and the reference lengths are written by host copies ordered
@@ -662,12 +665,13 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
         store_elem(static_cast<T*>(p.o) + (size_t)item.bh * D + dd, acc / Ls);
       } else if (p.cluster_merge) {
         // this CTA's partial into slot `rank` of the cluster leader's buffer
-        const uint32_t slot = cluster_map(smem_u32(cl_buf + (size_t)cluster_rank() * (D + 4)), 0);
-        st_cluster_f32(slot + 4u * dd, acc);
+        float* mine = cl_buf + (size_t)cluster_rank() * (D + 4);
+        mine[dd] = acc;
         if (dd == 0) {
-          st_cluster_f32(slot + 4u * D, M);
-          st_cluster_f32(slot + 4u * (D + 1), Ls);
+          mine[D] = M;
+          mine[D + 1] = Ls;
         }
+        fence_proxy_async_smem();
       } else {
         float* P = p.partials + (size_t)item.part * (D + 4);
         P[dd] = acc;
@@ -682,7 +686,16 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
     if (p.cluster_merge) {
       // one item per CTA: arrive on the leader's barrier with release at
       // cluster scope (after the barrier, so it covers every thread's stores)
-      if (tid == 0 && item_at(it0).nparts > 1) mbar_arrive_remote_release(cluster_map(cl_bar, 0));
+      if (tid == 0 && item_at(it0).nparts > 1) {
+        const uint32_t rank = cluster_rank();
+        if (rank == 0) {
+          mbar_arrive_expect_tx(cl_bar, (kDecodeCluster - 1) * (D + 4) * 4);
+        } else {
+          const uint32_t src = smem_u32(cl_buf + (size_t)rank * (D + 4));
+          bulk_s2cluster(cluster_map(src, 0), src, (D + 4) * 4, cluster_map(cl_bar, 0));
+          bulk_commit();
+        }
+      }
       continue;
     }
     // Tickets of the batch's split items right away: one release fence
@@ -763,6 +776,7 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
   }
 
   if (tid == 0) RSWA_STAMP(5);
+  if (p.cluster_merge && tid == 0) bulk_wait_read();  // the partial has left this CTA's shared memory
   if (APPEND && tid == 0 && launch_ticket == (int)gridDim.x - 1) {
     fence_acq_rel_gpu();
     if (p.full_mode && T0 + 1 > p.T_cap) flag_error(p.err, kErrCapacity);
