@@ -60,29 +60,6 @@ static bool dtype_ok(rswa_dtype t) { return t == RSWA_F32 || t == RSWA_BF16; }
 
 namespace rswa {
 
-bool encode_decode_cache_map(CUtensorMap* m, const void* base, unsigned long long rows) {
-  typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  });
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {128, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {256};
-  const cuuint32_t box[2] = {64, 32};
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 unsigned long long current_context_id() {
   typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
   static CtxGetIdFn fn = nullptr;
@@ -155,7 +132,6 @@ struct rswa_ctx {
   bool cluster_plan;          // the current plan merges each slab inside one cluster
   std::vector<DecodeItem> items;
   std::vector<int32_t> cta_begin;
-  CUtensorMap tmK, tmV;       // bf16, d = 128: the caches' TMA maps
 };
 
 static int32_t* ws_i32(rswa_ctx* c, size_t off) { return reinterpret_cast<int32_t*>(c->ws + off); }
@@ -394,13 +370,6 @@ extern "C" rswa_status rswa_init(rswa_handle* out, rswa_mode mode, int L_m_cap, 
   const char* plan = getenv("RSWA_DECODE_PLAN");  // "span": never use the cluster plan
   if (plan && strcmp(plan, "span") == 0) c->max_clusters = 0;
   c->cluster_plan = false;
-  if (dtype == RSWA_BF16 && d == 128) {
-    const unsigned long long rows = (unsigned long long)batch * H * c->S_cap;
-    if (!encode_decode_cache_map(&c->tmK, k_cache, rows) || !encode_decode_cache_map(&c->tmV, v_cache, rows)) {
-      delete c;
-      return fail(RSWA_ERR_CUDA, "rswa_init: cannot encode the caches' tensor maps");
-    }
-  }
   cudaError_t e = cudaMemsetAsync(c->ws, 0, lay.total, c->stream);
   if (e != cudaSuccess) {
     delete c;
@@ -622,8 +591,6 @@ static rswa_status run_decode(rswa_ctx* c, const void* k, const void* v, const v
   if (rswa_status st = use_device(c)) return st;
   if (rswa_status st = ensure_plan(c, c->T_host + (append ? 1 : 0))) return st;
   DecodeParams p;
-  p.tmK = c->tmK;
-  p.tmV = c->tmV;
   p.kc = c->kc;
   p.vc = c->vc;
   p.kc_w = c->kc;

@@ -89,11 +89,7 @@ struct DecTraits {
   static constexpr int kRPI = 32 / kLPR;               // rows per warp-wide load
   static constexpr int kNV = 8;                        // warp-wide loads per K (or V) part
   static constexpr int kStageRows = 32;                // rows per copied stage
-  // bf16, d = 128: one warp takes a whole 32-row stage, one key row per lane
-  // (stages land 128-byte swizzled by TMA, so lanes read different rows
-  // without bank conflicts); the other types split a stage over warps.
-  static constexpr bool kRowLane = std::is_same<T, __nv_bfloat16>::value && D == 128;
-  static constexpr int kWarpRows = kRowLane ? kStageRows : kNV * kRPI;  // 32 (bf16 d=128), 32 (bf16 d=64), 8 (f32 d=128)
+  static constexpr int kWarpRows = kNV * kRPI;         // 16 (bf16 d=128), 32 (bf16 d=64), 8 (f32 d=128)
   static constexpr int kSplit = kStageRows / kWarpRows;  // warps sharing a stage
   static constexpr int kStageBytes = kStageRows * kRowBytes;  // K or V part
   static constexpr int kW = 12;                        // consumer warps
@@ -115,8 +111,7 @@ struct DecTraits {
   // cluster merge: the leader's mbarrier and partials[kDecodeCluster][D + 4]
   static constexpr size_t kClBarOffset = (kQOffset + 4 * (size_t)kPreItems * D + 15) / 16 * 16;
   static constexpr size_t kClBufOffset = kClBarOffset + 16;
-  // + slack to align the stage ring to 1024 bytes (the 128-byte swizzle atom)
-  static constexpr size_t kSmemBytes = kClBufOffset + 4 * (size_t)kDecodeCluster * (D + 4) + 1024;
+  static constexpr size_t kSmemBytes = kClBufOffset + 4 * (size_t)kDecodeCluster * (D + 4);
   // partials that fit in the stage ring when it doubles as merge buffer
   static constexpr int kMergeCap = (int)(kBarOffset / ((D + 4) * 4));
 };
@@ -170,22 +165,6 @@ __device__ __forceinline__ float fma2_bf16(uint32_t a, uint32_t b, float acc) {
   return acc;
 }
 
-// o[0..3] += v[0..3] * w for four bf16 values (two packed words, low half
-// first) and a bf16 weight (low half of w), float32 accumulation (each
-// product of two bf16 values is exact in float32).
-__device__ __forceinline__ void fma4_bf16(uint2 v, uint32_t w, float* o) {
-  asm("{.reg .b16 v0, v1, v2, v3, wl, wh;\n\t"
-      "mov.b32 {v0, v1}, %4;\n\t"
-      "mov.b32 {v2, v3}, %5;\n\t"
-      "mov.b32 {wl, wh}, %6;\n\t"
-      "fma.rn.f32.bf16 %0, v0, wl, %0;\n\t"
-      "fma.rn.f32.bf16 %1, v1, wl, %1;\n\t"
-      "fma.rn.f32.bf16 %2, v2, wl, %2;\n\t"
-      "fma.rn.f32.bf16 %3, v3, wl, %3;\n\t}"
-      : "+f"(o[0]), "+f"(o[1]), "+f"(o[2]), "+f"(o[3])
-      : "r"(v.x), "r"(v.y), "r"(w));
-}
-
 // ---- thread-block cluster helpers (cluster-merge plan)
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
@@ -230,15 +209,6 @@ __device__ __forceinline__ void bulk_s2cluster(uint32_t dst, uint32_t src, uint3
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-// One box of a 2-D tensor map (coordinates: column, row) into shared memory,
-// completing its bytes on the mbarrier.
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
-      ::"r"(dst), "l"(map), "r"(c0), "r"(c1), "r"(bar)
-      : "memory");
-}
-
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void griddep_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -307,8 +277,7 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
   constexpr int W = Tr::kW, NT = Tr::kConsumerThreads;
   constexpr int RB = Tr::kRowBytes, SB = Tr::kStageBytes;
 
-  extern __shared__ __align__(128) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(128) uint8_t smem[];
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + Tr::kBarOffset);
   uint64_t* empty_bar = full_bar + NS;
   float* red_m = reinterpret_cast<float*>(smem + Tr::kRedOffset);  // [kBatch][W]
@@ -375,19 +344,9 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
     const size_t row = (size_t)item.bh * p.S_cap + item.row0 + (size_t)j * kStageRows;
     const uint32_t fb = smem_u32(&full_bar[slot]);
     uint8_t* dst = smem + (size_t)slot * 2 * SB;
-    if constexpr (Tr::kRowLane) {
-      // two 64-column boxes of 32 rows per tensor, always whole (rows past
-      // the slab are masked; past the tensor, zero-filled)
-      mbar_arrive_expect_tx(fb, 2 * SB);
-      tma_load_2d(smem_u32(dst), &p.tmK, 0, (int)row, fb);
-      tma_load_2d(smem_u32(dst + SB / 2), &p.tmK, 64, (int)row, fb);
-      tma_load_2d(smem_u32(dst + SB), &p.tmV, 0, (int)row, fb);
-      tma_load_2d(smem_u32(dst + SB + SB / 2), &p.tmV, 64, (int)row, fb);
-    } else {
-      mbar_arrive_expect_tx(fb, 2 * bytes);
-      bulk_g2s(smem_u32(dst), static_cast<const uint8_t*>(p.kc) + row * RB, bytes, fb);
-      bulk_g2s(smem_u32(dst + SB), static_cast<const uint8_t*>(p.vc) + row * RB, bytes, fb);
-    }
+    mbar_arrive_expect_tx(fb, 2 * bytes);
+    bulk_g2s(smem_u32(dst), static_cast<const uint8_t*>(p.kc) + row * RB, bytes, fb);
+    bulk_g2s(smem_u32(dst + SB), static_cast<const uint8_t*>(p.vc) + row * RB, bytes, fb);
     if (g == 0) RSWA_STAMP(2);
     ++g;
   };
@@ -558,20 +517,6 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
 #pragma unroll
     for (int e = 0; e < EPV; ++e) of[e] = 0.f;
     float m = -INFINITY, l = 0.f;
-    // Row per lane: the raw query (bf16 pairs), read chunk by chunk by every
-    // lane at once (a broadcast); this lane's 4 dims of it, and of the new
-    // token's k and v when the item holds its slot (loaded now, used when the
-    // warp meets the slot).
-    const uint4* qs = li < kPreItems ? reinterpret_cast<const uint4*>(s_q + li * D)
-                                     : reinterpret_cast<const uint4*>(static_cast<const T*>(p.q) + (size_t)item.bh * D);
-    uint2 q4 = make_uint2(0, 0), kn = make_uint2(0, 0), vn = make_uint2(0, 0);
-    if constexpr (Tr::kRowLane) {
-      q4 = reinterpret_cast<const uint2*>(qs)[lane];
-      if (APPEND && slot_row >= item.row0 && slot_row < item.row0 + item.rows) {
-        kn = *reinterpret_cast<const uint2*>(static_cast<const T*>(p.k_new) + (size_t)item.bh * D + 4 * lane);
-        vn = *reinterpret_cast<const uint2*>(static_cast<const T*>(p.v_new) + (size_t)item.bh * D + 4 * lane);
-      }
-    }
 
     // this warp group's stages of the item: global stage index = group (mod GR)
     const int j0 = (group - (int)(gctr % GR) + GR) % GR;
@@ -592,65 +537,7 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
       }
       // this warp's rows of the stage: [part_row, part_row + WR)
       const int nr = min(WR, live - j * kStageRows - part_row);  // may be <= 0: nothing to attend
-      if constexpr (Tr::kRowLane) {
-       if (nr > 0) {
-        // One key row per lane.  A stage is two 64-column boxes per tensor,
-        // 128-byte swizzled: 16-byte chunk c of row r sits at chunk
-        // (c ^ (r & 7)) of the row's 128 bytes, so the lanes' reads of one
-        // chunk column hit 8 different bank groups.
-        const int r_base = item.row0 + j * kStageRows;
-        const uint8_t* Kb = smem + (size_t)slot * 2 * SB;
-        const uint8_t* Vb = Kb + SB;
-        float d4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int c = 0; c < D / 8; ++c) {
-          const uint4 u = *reinterpret_cast<const uint4*>(Kb + (c >> 3) * (SB / 2) + lane * 128 + (((c & 7) ^ (lane & 7)) << 4));
-          const uint4 qc = qs[c];
-          d4[0] = fma2_bf16(qc.x, u.x, d4[0]);
-          d4[1] = fma2_bf16(qc.y, u.y, d4[1]);
-          d4[2] = fma2_bf16(qc.z, u.z, d4[2]);
-          d4[3] = fma2_bf16(qc.w, u.w, d4[3]);
-        }
-        float dot = (d4[0] + d4[1]) + (d4[2] + d4[3]);
-        // APPEND: the slot row holds the new token (the staged copy may
-        // predate it): its score from the new key, 4 dims per lane, and the
-        // new key and value stored into the slot.
-        const int slot_in = APPEND ? slot_row - r_base : -1;  // warp-uniform
-        if (APPEND && slot_in >= 0 && slot_in < nr) {
-          float part = fma2_bf16(q4.y, kn.y, fma2_bf16(q4.x, kn.x, 0.f));
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-          if (lane == slot_in) dot = part;
-          const size_t c_off = ((size_t)item.bh * p.S_cap + slot_row) * D + 4 * lane;
-          *reinterpret_cast<uint2*>(static_cast<T*>(p.kc_w) + c_off) = kn;
-          *reinterpret_cast<uint2*>(static_cast<T*>(p.vc_w) + c_off) = vn;
-        }
-        const float sc = lane < nr ? dot * p.scale_log2 : -INFINITY;
-        float mx = sc;
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        const float m_new = fmaxf(m, mx);  // finite: the stage has a valid row
-        const float corr = exp2f(m - m_new);
-        const float pr = lane < nr ? exp2f(sc - m_new) : 0.f;
-        l = l * corr + pr;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) of[e] *= corr;
-        // P.V with this lane's 4 output dims: chunk cv of every row, the
-        // weights broadcast as bf16 (the product rounds p to bf16, as a
-        // tensor-core P.V would)
-        const uint32_t pb = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(pr));
-        const int cv = lane >> 1;
-        const uint8_t* Vl = Vb + (cv >> 3) * (SB / 2) + (lane & 1) * 8;
-#pragma unroll 8
-        for (int rr = 0; rr < nr; ++rr) {
-          const uint32_t w = __shfl_sync(0xffffffffu, pb, rr);
-          uint2 v = *reinterpret_cast<const uint2*>(Vl + rr * 128 + (((cv & 7) ^ (rr & 7)) << 4));
-          if (APPEND && rr == slot_in) v = vn;
-          fma4_bf16(v, w, of);
-        }
-        m = m_new;
-       }
-      } else if (nr > 0) {
+      if (nr > 0) {
         const int r_base = item.row0 + j * kStageRows + part_row;
         const uint8_t* Ks = smem + (size_t)slot * 2 * SB + part_row * RB;
         const uint8_t* Vs = Ks + SB;
@@ -744,19 +631,14 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
     // ---- this warp's partial of item x: (m, l, o) into shared memory
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
-    if constexpr (Tr::kRowLane) {  // lane owns dims 4*lane .. 4*lane+3
 #pragma unroll
-      for (int e = 0; e < 4; ++e) red_o[(x * W + warp) * D + 4 * lane + e] = of[e];
-    } else {
+    for (int off = LPR; off < 32; off <<= 1) {
 #pragma unroll
-      for (int off = LPR; off < 32; off <<= 1) {
+      for (int e = 0; e < EPV; ++e) of[e] += __shfl_xor_sync(0xffffffffu, of[e], off);
+    }
+    if (grp == 0) {
 #pragma unroll
-        for (int e = 0; e < EPV; ++e) of[e] += __shfl_xor_sync(0xffffffffu, of[e], off);
-      }
-      if (grp == 0) {
-#pragma unroll
-        for (int e = 0; e < EPV; ++e) red_o[(x * W + warp) * D + sub * EPV + e] = of[e];
-      }
+      for (int e = 0; e < EPV; ++e) red_o[(x * W + warp) * D + sub * EPV + e] = of[e];
     }
     if (lane == 0) {
       red_m[x * W + warp] = m;

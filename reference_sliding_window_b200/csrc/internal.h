@@ -1,7 +1,6 @@
 // Internal interfaces between the C-ABI layer (api.cu) and the kernels.
 #pragma once
 
-#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -87,10 +86,6 @@ WorkspaceLayout workspace_layout(int B, int H, int d);
 enum ElemType : int { kF32 = 0, kBF16 = 1 };
 
 struct DecodeParams {
-  // bf16, D = 128: 2-D TMA maps of the caches, {D, B*H*S_cap} elements,
-  // boxes of 64 columns x 32 rows with 128-byte swizzle (the stages the
-  // row-per-lane consumers read without bank conflicts).
-  CUtensorMap tmK, tmV;
   const void* kc;        // cache [B][H][S_cap][D]
   const void* vc;
   void* kc_w;            // same buffers, written by the fused append
@@ -119,11 +114,6 @@ struct DecodeParams {
   float scale_log2;      // softmax scale * log2(e)
   unsigned long long* timing;  // profiling stamps (RSWA_TIMING builds), may be null
 };
-
-// Encodes the TMA map of one bf16 cache (rows x 128 elements, 256-byte row
-// pitch) as DecodeParams::tmK / tmV describe it.  False if the driver lacks
-// the entry point or rejects the map.
-bool encode_decode_cache_map(CUtensorMap* m, const void* base, unsigned long long rows);
 
 // Launch the split-K decode kernel (append: fused ring write + T advance).
 // CTAs per cluster in the cluster-merge plan.

@@ -172,11 +172,6 @@ extern "C" rswa_status rswa_decode_noalloc(const void* k_cache, const void* v_ca
     return na_fail(RSWA_ERR_CUDA, "staging the launch plan failed");
 
   DecodeParams p = {};
-  if (dtype == RSWA_BF16 && d == 128) {
-    const unsigned long long rows = (unsigned long long)batch * H * S_cap;
-    if (!encode_decode_cache_map(&p.tmK, k_cache, rows) || !encode_decode_cache_map(&p.tmV, v_cache, rows))
-      return na_fail(RSWA_ERR_CUDA, "cannot encode the caches' tensor maps");
-  }
   p.kc = k_cache;
   p.vc = v_cache;
   p.q = q;
