@@ -458,7 +458,7 @@ def run_decode(args, name, w, lens, T_target, steps, warmup, e2e_steps):
     `steps` steps are timed."""
     import torch
     import torch.distributed as dist
-    from reference_sliding_window_b200 import RSWA, append_decode_layers, synth
+    from reference_sliding_window_b200 import RSWA, LayerStep, append_decode_layers, synth
 
     world, rank, local = dist_env()
     dev = torch.device("cuda", local)
@@ -540,14 +540,15 @@ def run_decode(args, name, w, lens, T_target, steps, warmup, e2e_steps):
     host_out = torch.empty((K_e2e, R, B, H, d), dtype=dt, pin_memory=True)
     dev_in = torch.empty((R, 3, B, H, d), dtype=dt, device=dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    # per-layer views of the staging buffers, made once (as a model holds them)
-    kv_q = ([dev_in[r, 0] for r in range(R)], [dev_in[r, 1] for r in range(R)], [dev_in[r, 2] for r in range(R)])
+    # the step over the staging buffers, made once (as a model holds its buffers)
     with torch.cuda.stream(stream):
+        step_e2e = LayerStep(layers, [dev_in[r, 0] for r in range(R)], [dev_in[r, 1] for r in range(R)],
+                             [dev_in[r, 2] for r in range(R)], outs)
         torch.cuda.synchronize(dev)
         e0.record(stream)
         for i in range(K_e2e):
             dev_in.copy_(host_in[i % P], non_blocking=True)
-            append_decode_layers(layers, *kv_q, out=outs)
+            step_e2e()
             host_out[i].copy_(out, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize(dev)
@@ -560,7 +561,7 @@ def run_decode(args, name, w, lens, T_target, steps, warmup, e2e_steps):
     g.reset()
     if gt is not None:
         gt.reset()
-    del layers, pool, out, outs, views
+    del layers, pool, out, outs, views, step_e2e
     torch.cuda.empty_cache()
     s_el = 2 if w["dtype"] == "bf16" else 4
     return dict(name=name, R=R, K=steps, elapsed=elapsed, el_max=el_max, tok_sum=tok_sum, launches=launches,

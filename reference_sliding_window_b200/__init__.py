@@ -23,7 +23,7 @@ import torch
 from . import _native
 from ._native import MODE_FULL, MODE_RSWA, RSWAError, check
 
-__all__ = ["RSWA", "append_decode_layers", "masked_forward", "masked_forward_varlen", "RSWAError", "MODE_RSWA", "MODE_FULL", "library_version"]
+__all__ = ["RSWA", "LayerStep", "append_decode_layers", "masked_forward", "masked_forward_varlen", "RSWAError", "MODE_RSWA", "MODE_FULL", "library_version"]
 
 _DT = {torch.float32: _native.F32, torch.bfloat16: _native.BF16}
 
@@ -267,6 +267,36 @@ def append_decode_layers(layers: Sequence[RSWA], k: Sequence[torch.Tensor], v: S
         hs, R, P(*[t.data_ptr() for t in k]), P(*[t.data_ptr() for t in v]), P(*[t.data_ptr() for t in q]),
         P(*[t.data_ptr() for t in outs]), float(scale)))
     return outs
+
+
+class LayerStep:
+    """One decode step over fixed layer handles and fixed device buffers (a
+    model's per-layer k, v, q and output tensors, refilled in place every
+    step): the checks and the pointer arrays are done once, so each call is
+    a single C call of rswa_append_decode_layers."""
+
+    def __init__(self, layers: Sequence[RSWA], k: Sequence[torch.Tensor], v: Sequence[torch.Tensor],
+                 q: Sequence[torch.Tensor], out: Sequence[torch.Tensor], scale: float = 0.0):
+        R = len(layers)
+        if not (len(k) == len(v) == len(q) == len(out) == R) or R < 1:
+            raise ValueError("one k, v, q and out per layer")
+        for r, a in enumerate(layers):
+            a._vec("k", k[r])
+            a._vec("v", v[r])
+            a._vec("q", q[r])
+            a._vec("out", out[r])
+        P = C.c_void_p * R
+        self._layers = list(layers)
+        self._keep = (list(k), list(v), list(q), list(out))  # the tensors must outlive the step
+        self._args = (P(*[a._h.value for a in layers]), R, P(*[t.data_ptr() for t in k]),
+                      P(*[t.data_ptr() for t in v]), P(*[t.data_ptr() for t in q]),
+                      P(*[t.data_ptr() for t in out]), float(scale))
+        self._fn = _native.lib().rswa_append_decode_layers
+
+    def __call__(self) -> None:
+        for a in self._layers:
+            a._sync_stream()
+        check(self._fn(*self._args))
 
 
 def masked_forward(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, L_m: int, n: int,

@@ -17,7 +17,7 @@ import numpy as np
 import pytest
 import torch
 
-from reference_sliding_window_b200 import RSWA, RSWAError, append_decode_layers, synth
+from reference_sliding_window_b200 import RSWA, LayerStep, RSWAError, append_decode_layers, synth
 from tests import spikes
 from tests.gpu_util import compare_steps, make_attn, run_steps
 
@@ -77,7 +77,7 @@ def test_reference_in_chunks_equals_one_load(dtype, d):
     a.check()
 
 
-@pytest.mark.parametrize("graph", [False, True])
+@pytest.mark.parametrize("graph", [False, True, "step"])
 def test_layers_call_every_layer_matches_the_oracle(graph):
     """R = 4 layers of different reference lengths and the same batch; the
     queries spike on window edges at the sampled steps."""
@@ -92,7 +92,21 @@ def test_layers_call_every_layer_matches_the_oracle(graph):
     ins = [tuple(t.to(dev) for t in (c.k, c.v, c.q)) for c in cases]
     outs = [torch.empty_like(ins[r][2][0]) for r in range(R)]
     got = {r: {} for r in range(R)}
-    if not graph:
+    if graph == "step":  # fixed buffers refilled in place, one prebuilt C call per step
+        kin = [x[0][0].clone() for x in ins]
+        vin = [x[1][0].clone() for x in ins]
+        qin = [x[2][0].clone() for x in ins]
+        step = LayerStep(layers, kin, vin, qin, outs)
+        for t in range(1, T + 1):
+            for r in range(R):
+                kin[r].copy_(ins[r][0][t - 1])
+                vin[r].copy_(ins[r][1][t - 1])
+                qin[r].copy_(ins[r][2][t - 1])
+            step()
+            if t in steps:
+                for r in range(R):
+                    got[r][t] = outs[r].clone()
+    elif not graph:
         for t in range(1, T + 1):
             append_decode_layers(layers, [x[0][t - 1] for x in ins], [x[1][t - 1] for x in ins],
                                  [x[2][t - 1] for x in ins], out=outs)
