@@ -86,10 +86,9 @@ WorkspaceLayout workspace_layout(int B, int H, int d) {
   WorkspaceLayout w{};
   size_t off = 0;
   w.err = off;
-  w.done = off + 4;
   off = 256;
   w.T = off;
-  off = align_up(off + 4, 256);
+  off = align_up(off + 4 * (size_t)kStepSlots, 256);
   w.Lm = off;
   off = align_up(off + 4 * (size_t)B, 256);
   w.chunk = off;
@@ -172,7 +171,8 @@ static void make_plan(rswa_ctx* c) {
     }
   }
   const int Gc = nbh * kDecodeCluster;
-  c->cluster_plan = nbh <= c->max_clusters && Gc <= c->lay.max_ctas && Gc <= c->lay.items_cap;
+  c->cluster_plan =
+      nbh <= c->max_clusters && Gc <= c->lay.max_ctas && Gc <= c->lay.items_cap && Gc <= kStepSlots;
   if (c->cluster_plan) {
     c->items.clear();
     c->cta_begin.assign(Gc + 1, 0);
@@ -197,6 +197,7 @@ static void make_plan(rswa_ctx* c) {
     c->n_ctas = Gc;
     return;
   }
+  static_assert(kMinMergeCap / 2 <= kStepSlots, "a span-plan grid must fit the step-counter copies");
   const int G = (int)std::min<long long>(std::min(std::min(c->num_sms, c->lay.max_ctas), kMinMergeCap / 2), total);
   c->items.clear();
   c->cta_begin.assign(G + 1, 0);
@@ -412,7 +413,7 @@ extern "C" rswa_status rswa_load_reference(rswa_handle h, const void* K_ref, con
   RSWA_CUDA(cudaMemcpyAsync(h->ws + h->lay.Lm, h->Lm.data(), 4 * (size_t)h->B, cudaMemcpyHostToDevice,
                             h->stream),
             "upload reference lengths");
-  RSWA_CUDA(cudaMemsetAsync(h->ws + h->lay.T, 0, 4, h->stream), "reset step counter");
+  RSWA_CUDA(cudaMemsetAsync(h->ws + h->lay.T, 0, 4 * kStepSlots, h->stream), "reset step counter");
   if (rswa_status st = upload_plan(h)) return st;
   LoadRefParams p;
   p.kc = h->kc;
@@ -461,7 +462,7 @@ extern "C" rswa_status rswa_load_reference_chunk(rswa_handle h, const void* K, c
             "upload reference lengths");
   RSWA_CUDA(cudaMemcpyAsync(h->ws + h->lay.chunk, rows, 4 * (size_t)h->B, cudaMemcpyHostToDevice, h->stream),
             "upload chunk rows");
-  RSWA_CUDA(cudaMemsetAsync(h->ws + h->lay.T, 0, 4, h->stream), "reset step counter");
+  RSWA_CUDA(cudaMemsetAsync(h->ws + h->lay.T, 0, 4 * kStepSlots, h->stream), "reset step counter");
   if (all) {
     h->plan_window = h->mode == RSWA_MODE_RSWA ? h->n : std::min(h->T_cap, 64);
     make_plan(h);
@@ -613,7 +614,6 @@ static rswa_status run_decode(rswa_ctx* c, const void* k, const void* v, const v
   p.cta_begin = reinterpret_cast<const int32_t*>(c->ws + c->lay.cta_begin);
   p.partials = reinterpret_cast<float*>(c->ws + c->lay.partials);
   p.tickets = ws_i32(c, c->lay.tickets);
-  p.done = ws_i32(c, c->lay.done);
   p.err = ws_i32(c, c->lay.err);
   const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)c->d);
   p.scale_log2 = sc * 1.4426950408889634f;
@@ -739,7 +739,7 @@ extern "C" rswa_status rswa_reset(rswa_handle h) {
   if (rswa_status st = check_handle(h)) return st;
   if (!h->loaded) return fail(RSWA_ERR_STATE, "rswa_reset: no reference loaded");
   if (rswa_status st = use_device(h)) return st;
-  RSWA_CUDA(cudaMemsetAsync(h->ws + h->lay.T, 0, 4, h->stream), "reset step counter");
+  RSWA_CUDA(cudaMemsetAsync(h->ws + h->lay.T, 0, 4 * kStepSlots, h->stream), "reset step counter");
   h->T_host = 0;
   return RSWA_OK;
 }
@@ -919,8 +919,10 @@ extern "C" rswa_status rswa_masked_forward_fill(rswa_handle h, const void* Q, co
   if (rswa_status st = upload_plan(h)) return st;
   if (h->dtype == RSWA_BF16 && h->d == 128) {
     // One tensor-core launch computes O and writes the cache rows.
-    int32_t T0_dev = T0;
-    RSWA_CUDA(cudaMemcpyAsync(h->ws + h->lay.T, &T0_dev, 4, cudaMemcpyHostToDevice, h->stream), "set step counter");
+    // (pageable source: the copy is staged before the call returns)
+    std::vector<int32_t> T0_dev(kStepSlots, T0);
+    RSWA_CUDA(cudaMemcpyAsync(h->ws + h->lay.T, T0_dev.data(), 4 * kStepSlots, cudaMemcpyHostToDevice, h->stream),
+              "set step counter");
     MaskedParams p;
     p.Q = Q;
     p.K = K;

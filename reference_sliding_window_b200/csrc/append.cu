@@ -16,8 +16,8 @@
 namespace rswa {
 
 // One CTA: read the step counter T once, write the B*H new rows of k and v
-// into their slots, then advance T.  Only this CTA touches T, so there is no
-// race.  (Not the hot path: decoding uses the fused kernel.)
+// into their slots, then advance every copy of T.  Only this CTA touches T,
+// so there is no race.  (Not the hot path: decoding uses the fused kernel.)
 __global__ void __launch_bounds__(256) append_kernel(const __grid_constant__ AppendParams p) {
   __shared__ int s_T, s_ok;
   if (threadIdx.x == 0) {
@@ -45,7 +45,8 @@ __global__ void __launch_bounds__(256) append_kernel(const __grid_constant__ App
     }
   }
   __syncthreads();
-  if (threadIdx.x == 0 && s_ok) *p.T = Tn;
+  if (s_ok)
+    for (int e = threadIdx.x; e < kStepSlots; e += blockDim.x) p.T[e] = Tn;
 }
 
 // grid.y = B*H slabs, grid.x covers max_len rows x vectors; copies rows
@@ -106,7 +107,8 @@ __global__ void __launch_bounds__(256) load_packed_kernel(const __grid_constant_
     *reinterpret_cast<uint4*>(kd + dof) = *reinterpret_cast<const uint4*>(ks + so);
     *reinterpret_cast<uint4*>(vd + dof) = *reinterpret_cast<const uint4*>(vs + so);
   }
-  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *p.T = p.T0;
+  if (blockIdx.x == 0 && blockIdx.y == 0)
+    for (int e = threadIdx.x; e < kStepSlots; e += blockDim.x) p.T[e] = p.T0;
   // Same contract as load_reference_kernel: decode kernels may copy
   // reference rows before their dependency wait.
   __threadfence();

@@ -18,7 +18,7 @@ struct LoadPackedParams {
   int B, H, S_cap, row_bytes, seq_stride;
   int n, T0, full_mode;
   const int32_t* Lm;   // device [B]
-  int32_t* T;          // device step counter, set to T0
+  int32_t* T;          // device step counter (kStepSlots copies), all set to T0
 };
 cudaError_t launch_load_packed(const LoadPackedParams& p, int max_rows, cudaStream_t stream);
 

@@ -21,8 +21,8 @@
 //   barrier set-up, the plan and reference lengths (host-written) staged in
 //   shared memory, copies of the leading stages made only of reference rows
 //   (written only by the reference load, whose kernel fences before it
-//   retires), and an L2 prefetch of the remaining rows.  The ring rows, q
-//   and the step counter are read after the wait.  The next kernel may
+//   retires), and an L2 prefetch of the remaining rows, q and the new rows.
+//   The ring rows, q and the step counter are read after the wait.  The next kernel may
 //   launch as soon as this one has started.
 // * One producer lane streams the stages into a ring of shared-memory
 //   buffers with bulk async copies (cp.async.bulk, completion on mbarriers).
@@ -54,9 +54,10 @@
 //   barrier expects the other CTAs' bytes, waits and merges.
 // * APPEND: the consumer that meets the slot row substitutes the new k/v
 //   (the staged copy of that row may predate the write) and stores them into
-//   the slot.  Each CTA reads the step counter T once and then takes a
-//   launch ticket; the CTA with the last ticket knows every CTA has read T
-//   and advances it.  One kernel per decode step, replayable in a CUDA graph.
+//   the slot.  The step counter T has one copy per CTA: each CTA reads its
+//   own copy and at its end writes T + 1 into copies no other CTA of the
+//   launch reads (kStepSlots in internal.h), so advancing T costs no atomic
+//   and no fence.  One kernel per decode step, replayable in a CUDA graph.
 // * Every wait is bounded; a timeout sets the device error word and the
 //   kernel finishes without trapping.
 
@@ -296,6 +297,7 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
+  static_assert(kStepSlots <= NT, "one step-counter copy per consumer thread at most");
   if (threadIdx.x == 0) {
     RSWA_STAMP(0);
     for (int s = 0; s < NS; ++s) {
@@ -393,6 +395,19 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
     RSWA_STAMP(12);
   }
 #endif
+  // q, the new rows and this CTA's copy of T into L2 (coherent: a value the
+  // previous kernel still writes is fetched again when read after the wait).
+  if (warp == W && lane == 1) {
+    for (int i = 0; i < n_pre; ++i) {
+      const size_t off = (size_t)s_items[i].bh * D * sizeof(T);
+      bulk_prefetch_l2(static_cast<const uint8_t*>(p.q) + off, D * sizeof(T));
+      if (APPEND) {
+        bulk_prefetch_l2(static_cast<const uint8_t*>(p.k_new) + off, D * sizeof(T));
+        bulk_prefetch_l2(static_cast<const uint8_t*>(p.v_new) + off, D * sizeof(T));
+      }
+    }
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p.T + (APPEND ? blockIdx.x : 0)));
+  }
   griddep_wait();  // everything below may read what the previous kernel wrote
   if (threadIdx.x == 0) RSWA_STAMP(1);
 
@@ -428,15 +443,22 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
   }
 
   // ------------------------------------------------------------ consumers
-  // The step counter and the queries of the staged items are outputs of
-  // earlier kernels: one round of independent loads.
-  if (threadIdx.x == 0) *s_T = ld_cg(p.T);
+  // The step counter (this CTA's copy) and the queries of the staged items
+  // are outputs of earlier kernels: one round of independent loads, every
+  // load issued before any result is used.
   {
     constexpr int VPR = D / EPV;  // 16-byte vectors per query row
-    for (int x = threadIdx.x; x < n_pre * VPR; x += NT) {
+    static_assert(kPreItems * VPR <= NT, "one query vector per consumer thread");
+    const int x = threadIdx.x;
+    int t_val = 0;
+    if (x == 0) t_val = ld_cg(p.T + (APPEND ? blockIdx.x : 0));
+    uint4 qu = make_uint4(0, 0, 0, 0);
+    if (x < n_pre * VPR)
+      qu = *reinterpret_cast<const uint4*>(static_cast<const T*>(p.q) + (size_t)s_items[x / VPR].bh * D +
+                                           (x % VPR) * EPV);
+    if (x == 0) *s_T = t_val;
+    if (x < n_pre * VPR) {
       const int i = x / VPR, v = x % VPR;
-      const uint4 qu =
-          *reinterpret_cast<const uint4*>(static_cast<const T*>(p.q) + (size_t)s_items[i].bh * D + v * EPV);
       if (kMixed) {
         reinterpret_cast<uint4*>(s_q + i * D)[v] = qu;  // raw bf16
       } else {
@@ -454,12 +476,6 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
   }
   const int T0 = *s_T;
   const int T_step = T0 + (APPEND ? 1 : 0);  // outputs in the cache for this step
-  // Launch ticket, taken right after the read of T but only looked at at the
-  // end: the CTA holding the last ticket knows every CTA has read T, so it
-  // may advance T (the others keep their copy).
-  // (Relaxed: this thread's read of T has already returned and been used.)
-  int launch_ticket = 0;
-  if (APPEND && threadIdx.x == 0) launch_ticket = atomic_add_relaxed(p.done, 1);
   const int group = warp / Tr::kSplit;            // stage group of this warp
   const int part_row = (warp % Tr::kSplit) * WR;  // its first row inside a stage
   const int grp = lane / LPR;   // which of the RPI rows of a warp-wide load
@@ -544,20 +560,28 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
         float part[NV];
         int sub_k = -1;
         uint4 vsub = make_uint4(0, 0, 0, 0);
+        uint4 ku[NV];
 #pragma unroll
-        for (int k = 0; k < NV; ++k) {
-          const int row = k * RPI + grp;
-          uint4 u = *reinterpret_cast<const uint4*>(Ks + row * RB + sub * 16);
-          if (APPEND && r_base + row == slot_row) {
+        for (int k = 0; k < NV; ++k) ku[k] = *reinterpret_cast<const uint4*>(Ks + (k * RPI + grp) * RB + sub * 16);
+        if (APPEND) {
+          const int rel = slot_row - r_base - grp;
+          if (rel >= 0 && rel < NV * RPI && rel % RPI == 0) {
             // The new token: use its k/v from the inputs and store it into its slot.
+            sub_k = rel / RPI;
             const size_t in_off = (size_t)item.bh * D + sub * EPV;
             const size_t c_off = ((size_t)item.bh * p.S_cap + slot_row) * D + sub * EPV;
-            u = *reinterpret_cast<const uint4*>(static_cast<const T*>(p.k_new) + in_off);
+            const uint4 kn = *reinterpret_cast<const uint4*>(static_cast<const T*>(p.k_new) + in_off);
             vsub = *reinterpret_cast<const uint4*>(static_cast<const T*>(p.v_new) + in_off);
-            *reinterpret_cast<uint4*>(static_cast<T*>(p.kc_w) + c_off) = u;
+            *reinterpret_cast<uint4*>(static_cast<T*>(p.kc_w) + c_off) = kn;
             *reinterpret_cast<uint4*>(static_cast<T*>(p.vc_w) + c_off) = vsub;
-            sub_k = k;
+#pragma unroll
+            for (int k = 0; k < NV; ++k)
+              if (k == sub_k) ku[k] = kn;
           }
+        }
+#pragma unroll
+        for (int k = 0; k < NV; ++k) {
+          const uint4 u = ku[k];
           float acc = 0.f;
           if (kMixed) {
             acc = fma2_bf16(qraw.x, u.x, acc);
@@ -594,30 +618,39 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
         const bool owner = sub < NV;  // one lane per row adds to the sum
         if (gs == 0 && lane == 0) RSWA_CYC(4);
         const float sc = valid ? (kMixed ? part[0] * p.scale_log2 : part[0]) : -INFINITY;
-        float mx = sc;
+        // Lazy running maximum: exponents stay <= 2^8 over the maximum in use,
+        // so the maximum is reduced (and o, l rescaled) only when a score
+        // exceeds it by more than 8 (always on a warp's first part).
+        if (__any_sync(0xffffffffu, sc > m + 8.f)) {
+          float mx = sc;
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        const float m_new = fmaxf(m, mx);  // finite: the stage has a valid row
-        const float corr = exp2f(m - m_new);
-        const float pr = valid ? exp2f(sc - m_new) : 0.f;
-        l = l * corr + (owner ? pr : 0.f);
+          for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+          const float m_new = fmaxf(m, mx);  // finite: the stage has a valid row
+          const float corr = exp2f(m - m_new);
+          l *= corr;
+#pragma unroll
+          for (int e = 0; e < EPV; ++e) of[e] *= corr;
+          m = m_new;
+        }
+        const float pr = valid ? exp2f(sc - m) : 0.f;
+        l += owner ? pr : 0.f;
         if (gs == 0 && lane == 0) RSWA_CYC(5);
+        uint4 vu[NV];
+        float pk[NV];
 #pragma unroll
-        for (int e = 0; e < EPV; ++e) of[e] *= corr;
+        for (int k = 0; k < NV; ++k) vu[k] = *reinterpret_cast<const uint4*>(Vs + (k * RPI + grp) * RB + sub * 16);
+#pragma unroll
+        for (int k = 0; k < NV; ++k) pk[k] = __shfl_sync(0xffffffffu, pr, grp * LPR + k);
 #pragma unroll
         for (int k = 0; k < NV; ++k) {
-          const int row = k * RPI + grp;
-          const float pk = __shfl_sync(0xffffffffu, pr, grp * LPR + k);
-          if (row < nr) {
-            uint4 u = *reinterpret_cast<const uint4*>(Vs + row * RB + sub * 16);
-            if (APPEND && k == sub_k) u = vsub;
+          if (APPEND && k == sub_k) vu[k] = vsub;
+          if (k * RPI + grp < nr) {
             float f[EPV];
-            Vec16<T>::unpack(u, f);
+            Vec16<T>::unpack(vu[k], f);
 #pragma unroll
-            for (int e = 0; e < EPV; ++e) of[e] = fmaf(pk, f[e], of[e]);
+            for (int e = 0; e < EPV; ++e) of[e] = fmaf(pk[k], f[e], of[e]);
           }
         }
-        m = m_new;
       }
       if (gs == 0 && lane == 0) {
         RSWA_STAMP(9);
@@ -777,12 +810,13 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
 
   if (tid == 0) RSWA_STAMP(5);
   if (p.cluster_merge && tid == 0) bulk_wait_read();  // the partial has left this CTA's shared memory
-  if (APPEND && tid == 0 && launch_ticket == (int)gridDim.x - 1) {
-    fence_acq_rel_gpu();
-    if (p.full_mode && T0 + 1 > p.T_cap) flag_error(p.err, kErrCapacity);
-    else *p.T = T0 + 1;
-    *p.done = 0;
+  // Advance T: copies blockIdx.x, blockIdx.x + grid, ... (kStepSlots <= NT,
+  // one store per thread), none of which another CTA of this launch reads.
+  if (APPEND && !(p.full_mode && T0 + 1 > p.T_cap)) {
+    const int e = blockIdx.x + tid * gridDim.x;
+    if (e < kStepSlots) p.T[e] = T0 + 1;
   }
+  if (APPEND && tid == 0 && blockIdx.x == 0 && p.full_mode && T0 + 1 > p.T_cap) flag_error(p.err, kErrCapacity);
   if (tid == 0) RSWA_STAMP(6);
 }
 

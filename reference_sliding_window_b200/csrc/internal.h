@@ -65,11 +65,19 @@ struct DecodeItem {
   int32_t part_first, nparts, last, pad;
 };
 
+// The step counter T is kept as kStepSlots equal copies.  A fused
+// append+decode launch has every CTA read its own copy and, when done, write
+// T + 1 into the copies c, c + grid, c + 2*grid, ...: no CTA reads a copy
+// that another CTA of the same launch writes, so no ticket or fence is needed
+// to advance T.  Every other writer sets all copies; readers on the host use
+// copy 0.  A decode grid never exceeds kStepSlots CTAs.
+constexpr int kStepSlots = 256;
+
 // Device workspace layout (byte offsets from the workspace base).
 struct WorkspaceLayout {
   size_t err;        // int32: device error word
-  size_t done;       // int32: end-of-launch ticket (fused append+decode)
-  size_t T;          // int32: outputs appended so far (every sequence advances together)
+  size_t T;          // int32[kStepSlots]: outputs appended so far (every sequence advances
+                     // together), one equal copy per decode CTA
   size_t Lm;         // int32[B]: reference rows
   size_t chunk;      // int32[B]: rows of the reference chunk being appended
   size_t tickets;    // int32[B*H]: split-K tickets
@@ -100,13 +108,12 @@ struct DecodeParams {
   int T_cap;             // FULL mode capacity
   int n_ctas;            // grid size; CTA c runs items [cta_begin[c], cta_begin[c+1])
   int n_items_total;
-  int32_t* T;            // scalar step counter
+  int32_t* T;            // step counter, kStepSlots equal copies (CTA c reads copy c)
   const int32_t* Lm;     // [B]
   const DecodeItem* items;
   const int32_t* cta_begin;
   float* partials;
   int32_t* tickets;
-  int32_t* done;
   int32_t* err;
   int ref_stable;        // 1: the reference rows are final (see decode.cu); 0: read after the wait
   int cluster_merge;     // 1: the kDecodeCluster CTAs of a slab form a cluster and merge in
@@ -136,7 +143,7 @@ struct AppendParams {
   const void* k_new;
   const void* v_new;
   int B, H, S_cap, row_bytes, n, full_mode, T_cap;
-  int32_t* T;
+  int32_t* T;  // step counter (kStepSlots copies): copy 0 read, all advanced
   const int32_t* Lm;
   int32_t* err;
 };

@@ -190,7 +190,6 @@ extern "C" rswa_status rswa_decode_noalloc(const void* k_cache, const void* v_ca
   p.cta_begin = reinterpret_cast<const int32_t*>(scratch + kNaCtaBegin);
   p.partials = reinterpret_cast<float*>(scratch + kNaPartials);
   p.tickets = reinterpret_cast<int32_t*>(scratch + kNaTickets);
-  p.done = reinterpret_cast<int32_t*>(scratch + kNaDone);
   p.err = reinterpret_cast<int32_t*>(scratch + kNaErr);
   const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)d);
   p.scale_log2 = sc * 1.4426950408889634f;
