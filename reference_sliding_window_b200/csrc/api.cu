@@ -12,6 +12,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <map>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -129,6 +130,7 @@ struct rswa_ctx {
   int n_ctas;
   int max_clusters;           // resident clusters of kDecodeCluster decode CTAs
   bool cluster_plan;          // the current plan merges each slab inside one cluster
+  std::vector<int32_t> cl_rows, cl_lm;  // cluster plan: planned rows and L_m per slab
   std::vector<DecodeItem> items;
   std::vector<int32_t> cta_begin;
 };
@@ -171,9 +173,12 @@ static void make_plan(rswa_ctx* c) {
     }
   }
   const int Gc = nbh * kDecodeCluster;
-  c->cluster_plan =
-      nbh <= c->max_clusters && Gc <= c->lay.max_ctas && Gc <= c->lay.items_cap && Gc <= kStepSlots;
+  c->cluster_plan = nbh <= c->max_clusters && nbh <= kClusterPlanMaxSlabs && Gc <= c->lay.max_ctas &&
+                    Gc <= c->lay.items_cap && Gc <= kStepSlots;
   if (c->cluster_plan) {
+    c->cl_rows = rows;
+    c->cl_lm.assign(nbh, 0);
+    for (int bh = 0; bh < nbh; ++bh) c->cl_lm[bh] = c->Lm[bh / c->H];
     c->items.clear();
     c->cta_begin.assign(Gc + 1, 0);
     for (int bh = 0; bh < nbh; ++bh) {
@@ -380,7 +385,35 @@ extern "C" rswa_status rswa_init(rswa_handle* out, rswa_mode mode, int L_m_cap, 
   return RSWA_OK;
 }
 
-extern "C" void rswa_destroy(rswa_handle h) { delete h; }
+// The handle of the decode this library last launched on each (device,
+// stream).  A decode may copy ring rows before its dependency wait only if
+// the previous kernel on its stream is not a decode of the same handle (the
+// decode kernel's prologue states why that suffices).  Any kernel launched in
+// between, by this library or not, only makes the answer conservative.
+// cudaStreamPerThread names a different stream on each host thread, so it
+// always answers "same handle".
+static std::mutex g_last_decode_mu;
+static std::map<std::pair<int, cudaStream_t>, const rswa_ctx*> g_last_decode;
+
+static bool previous_decode_is(const rswa_ctx* c) {
+  if (c->stream == cudaStreamPerThread) return true;
+  std::lock_guard<std::mutex> lock(g_last_decode_mu);
+  const auto key = std::make_pair(c->device, c->stream);
+  auto it = g_last_decode.find(key);
+  const bool same = it != g_last_decode.end() && it->second == c;
+  g_last_decode[key] = c;
+  return same;
+}
+
+extern "C" void rswa_destroy(rswa_handle h) {
+  if (!h) return;
+  {
+    std::lock_guard<std::mutex> lock(g_last_decode_mu);
+    for (auto it = g_last_decode.begin(); it != g_last_decode.end();)
+      it = it->second == h ? g_last_decode.erase(it) : std::next(it);
+  }
+  delete h;
+}
 
 extern "C" rswa_status rswa_set_stream(rswa_handle h, void* stream) {
   if (rswa_status st = check_handle(h)) return st;
@@ -575,6 +608,7 @@ extern "C" rswa_status rswa_append(rswa_handle h, const void* k, const void* v) 
 
 // Profiling aid: per-CTA timestamp buffer used by RSWA_TIMING builds.
 static unsigned long long* g_timing = nullptr;
+
 #ifdef RSWA_TIMING
 extern "C" void rswa_debug_set_timing(void* buf) { g_timing = static_cast<unsigned long long*>(buf); }
 #endif
@@ -619,14 +653,21 @@ static rswa_status run_decode(rswa_ctx* c, const void* k, const void* v, const v
   p.scale_log2 = sc * 1.4426950408889634f;
   p.timing = g_timing;
   p.cluster_merge = c->cluster_plan ? 1 : 0;
-  // Only rswa_load_reference writes the reference rows, and its kernel
-  // fences its writes before retiring, so every later decode may copy them
-  // before its dependency wait.
+  // Reference rows may always be copied before the dependency wait, ring
+  // rows unless the previous kernel on the stream is a decode of this handle
+  // (decode.cu states the argument).
 #ifdef RSWA_NO_EARLY_COPY
   p.ref_stable = 0;
+  p.ring_early = 0;
 #else
   p.ref_stable = 1;
+  p.ring_early = previous_decode_is(c) ? 0 : 1;
 #endif
+  if (c->cluster_plan)
+    for (int bh = 0; bh < c->B * c->H; ++bh) {
+      p.cl_rows[bh] = c->cl_rows[bh];
+      p.cl_lm[bh] = c->cl_lm[bh];
+    }
   const int grid = c->n_ctas;
   RSWA_CUDA(launch_decode(c->dtype == RSWA_BF16 ? kBF16 : kF32, c->d, append, p, grid, c->stream),
             "decode kernel");

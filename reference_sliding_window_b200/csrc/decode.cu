@@ -19,11 +19,11 @@
 //   kDecodeCluster CTAs of cluster bh, one contiguous part each.
 // * Before waiting on the previous kernel (programmatic dependent launch):
 //   barrier set-up, the plan and reference lengths (host-written) staged in
-//   shared memory, copies of the leading stages made only of reference rows
-//   (written only by the reference load, whose kernel fences before it
-//   retires), and an L2 prefetch of the remaining rows, q and the new rows.
-//   The ring rows, q and the step counter are read after the wait.  The next kernel may
-//   launch as soon as this one has started.
+//   shared memory, copies of the leading stages (reference rows, and ring
+//   rows when the host allows it: see the prologue), and an L2 prefetch of
+//   the remaining rows, q and the new rows.  q, the new rows and the step
+//   counter are read after the wait.  The next kernel may launch once this
+//   one has passed its own wait.
 // * One producer lane streams the stages into a ring of shared-memory
 //   buffers with bulk async copies (cp.async.bulk, completion on mbarriers).
 // * Stage g (32 rows, counted over the launch) goes to consumer warp group
@@ -110,9 +110,13 @@ struct DecTraits {
   static constexpr size_t kLmOffset = kMetaOffset + sizeof(DecodeItem) * kPreItems;
   static constexpr size_t kQOffset = kLmOffset + 4 * kPreItems;
   // cluster merge: the leader's mbarrier and partials[kDecodeCluster][D + 4]
-  static constexpr size_t kClBarOffset = (kQOffset + 4 * (size_t)kPreItems * D + 15) / 16 * 16;
+  // fused append: the new key and value rows of the staged items, [kPreItems][row] each
+  static constexpr size_t kKnOffset = (kQOffset + 4 * (size_t)kPreItems * D + 15) / 16 * 16;
+  static constexpr size_t kVnOffset = kKnOffset + (size_t)kPreItems * kRowBytes;
+  static constexpr size_t kClBarOffset = (kVnOffset + (size_t)kPreItems * kRowBytes + 15) / 16 * 16;
   static constexpr size_t kClBufOffset = kClBarOffset + 16;
   static constexpr size_t kSmemBytes = kClBufOffset + 4 * (size_t)kDecodeCluster * (D + 4);
+  static_assert(kSmemBytes <= 227 * 1024, "dynamic shared memory above the per-CTA limit");
   // partials that fit in the stage ring when it doubles as merge buffer
   static constexpr int kMergeCap = (int)(kBarOffset / ((D + 4) * 4));
 };
@@ -290,6 +294,8 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
   DecodeItem* s_items = reinterpret_cast<DecodeItem*>(smem + Tr::kMetaOffset);
   int* s_lm = reinterpret_cast<int*>(smem + Tr::kLmOffset);
   float* s_q = reinterpret_cast<float*>(smem + Tr::kQOffset);
+  uint8_t* s_kn = smem + Tr::kKnOffset;
+  uint8_t* s_vn = smem + Tr::kVnOffset;
   const uint32_t cl_bar = smem_u32(smem + Tr::kClBarOffset);
   float* cl_buf = reinterpret_cast<float*>(smem + Tr::kClBufOffset);  // [kDecodeCluster][D + 4]
   float* merge_buf = reinterpret_cast<float*>(smem);  // the stage ring, once drained
@@ -314,20 +320,40 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
   // kernel.  So can an L2 prefetch of the rows this CTA will stream: L2 is
   // coherent, so a row the previous kernel still writes is simply fetched
   // again later.
-  const int it_begin = p.cta_begin[blockIdx.x];
-  const int it_end = p.cta_begin[blockIdx.x + 1];
+  // Cluster plan: one item per CTA, derived from the CTA index and the
+  // per-slab sizes in the parameters exactly as the host planner makes it,
+  // so no chain of dependent global loads delays the first copies.
+  const int it_begin = p.cluster_merge ? (int)blockIdx.x : p.cta_begin[blockIdx.x];
+  const int it_end = p.cluster_merge ? (int)blockIdx.x + 1 : p.cta_begin[blockIdx.x + 1];
   const int n_pre = min(it_end - it_begin, kPreItems);
   if ((int)threadIdx.x < n_pre) {
-    const DecodeItem item = p.items[it_begin + threadIdx.x];
+    DecodeItem item;
+    int lm;
+    if (p.cluster_merge) {
+      const int c = blockIdx.x, bh = c / kDecodeCluster, r = c % kDecodeCluster;
+      const int rows_bh = p.cl_rows[bh], S = (rows_bh + 31) / 32;
+      const int st0 = (int)((long long)S * r / kDecodeCluster), st1 = (int)((long long)S * (r + 1) / kDecodeCluster);
+      item.bh = bh;
+      item.row0 = st0 * 32;
+      item.rows = max(0, min(rows_bh, st1 * 32) - item.row0);
+      item.part = c;
+      item.part_first = bh * kDecodeCluster;
+      item.nparts = kDecodeCluster;
+      item.last = r == kDecodeCluster - 1;
+      item.pad = 0;
+      lm = p.cl_lm[bh];
+    } else {
+      item = p.items[it_begin + threadIdx.x];
+      lm = p.Lm[item.bh / p.H];
+    }
     s_items[threadIdx.x] = item;
-    s_lm[threadIdx.x] = p.Lm[item.bh / p.H];
+    s_lm[threadIdx.x] = lm;
   }
   __syncthreads();
   // Cluster-merge plan: the leader's barrier must be initialised before any
   // CTA of the cluster arrives on it.  Every thread passes here (no thread
   // has exited yet), so this hardware barrier cannot be left waiting.
   if (p.cluster_merge) cluster_sync_all();
-  griddep_launch_dependents();
   auto item_at = [&](int it) -> DecodeItem {
     const int li = it - it_begin;
     return li < kPreItems ? s_items[li] : p.items[it];
@@ -352,11 +378,16 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
     if (g == 0) RSWA_STAMP(2);
     ++g;
   };
-  // Reference rows are written only by the reference load, whose kernel
-  // fences its writes before it retires, so with ref_stable the leading
-  // stages made only of reference rows are copied before the dependency
-  // wait, into buffers that are still free (g < NS).  Output rows (the
-  // ring) may be written by the previous kernel and are copied after it.
+  // With ref_stable the leading stages made only of reference rows are
+  // copied before the dependency wait, into buffers that are still free
+  // (g < NS): only the cache loads and the prefill fill write them, and
+  // those kernels never let a dependent start before they retire.  With
+  // ring_early, leading stages that hold ring rows are copied early too.
+  // Ring rows are written by those kernels and by a fused append+decode,
+  // which lets the next kernel start only after its own dependency wait
+  // (above), so when this CTA runs, every decode before the previous kernel
+  // has retired; the host sets ring_early only when the previous kernel it
+  // launched on the stream was not a decode of this handle.
   if (warp == W && lane == 0 && p.ref_stable) {
     while (p_it < it_end && g < (uint32_t)NS) {
       const DecodeItem item = item_at(p_it);
@@ -367,7 +398,7 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
         continue;
       }
       const int nr = min(kStageRows, item.rows - p_j * kStageRows);
-      if (item.row0 + p_j * kStageRows + nr > lm_at(p_it, item)) break;
+      if (!p.ring_early && item.row0 + p_j * kStageRows + nr > lm_at(p_it, item)) break;
       issue(item, p_j);
       ++p_j;
     }
@@ -409,6 +440,10 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
     asm volatile("prefetch.global.L2 [%0];" ::"l"(p.T + (APPEND ? blockIdx.x : 0)));
   }
   griddep_wait();  // everything below may read what the previous kernel wrote
+  // Only now may the next kernel start: every kernel before this one has
+  // retired by then, which is what lets a decode copy ring rows before its
+  // own wait (prologue).
+  griddep_launch_dependents();
   if (threadIdx.x == 0) RSWA_STAMP(1);
 
   // ------------------------------------------------------------ producer
@@ -452,13 +487,22 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
     const int x = threadIdx.x;
     int t_val = 0;
     if (x == 0) t_val = ld_cg(p.T + (APPEND ? blockIdx.x : 0));
-    uint4 qu = make_uint4(0, 0, 0, 0);
-    if (x < n_pre * VPR)
-      qu = *reinterpret_cast<const uint4*>(static_cast<const T*>(p.q) + (size_t)s_items[x / VPR].bh * D +
-                                           (x % VPR) * EPV);
+    uint4 qu = make_uint4(0, 0, 0, 0), kn = qu, vn = qu;
+    if (x < n_pre * VPR) {
+      const size_t off = (size_t)s_items[x / VPR].bh * D + (x % VPR) * EPV;
+      qu = *reinterpret_cast<const uint4*>(static_cast<const T*>(p.q) + off);
+      if (APPEND) {  // the new rows, for the consumer that meets the slot row
+        kn = *reinterpret_cast<const uint4*>(static_cast<const T*>(p.k_new) + off);
+        vn = *reinterpret_cast<const uint4*>(static_cast<const T*>(p.v_new) + off);
+      }
+    }
     if (x == 0) *s_T = t_val;
     if (x < n_pre * VPR) {
       const int i = x / VPR, v = x % VPR;
+      if (APPEND) {
+        reinterpret_cast<uint4*>(s_kn + i * RB)[v] = kn;
+        reinterpret_cast<uint4*>(s_vn + i * RB)[v] = vn;
+      }
       if (kMixed) {
         reinterpret_cast<uint4*>(s_q + i * D)[v] = qu;  // raw bf16
       } else {
@@ -570,8 +614,14 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
             sub_k = rel / RPI;
             const size_t in_off = (size_t)item.bh * D + sub * EPV;
             const size_t c_off = ((size_t)item.bh * p.S_cap + slot_row) * D + sub * EPV;
-            const uint4 kn = *reinterpret_cast<const uint4*>(static_cast<const T*>(p.k_new) + in_off);
-            vsub = *reinterpret_cast<const uint4*>(static_cast<const T*>(p.v_new) + in_off);
+            uint4 kn;
+            if (li < kPreItems) {
+              kn = reinterpret_cast<const uint4*>(s_kn + li * RB)[sub];
+              vsub = reinterpret_cast<const uint4*>(s_vn + li * RB)[sub];
+            } else {
+              kn = *reinterpret_cast<const uint4*>(static_cast<const T*>(p.k_new) + in_off);
+              vsub = *reinterpret_cast<const uint4*>(static_cast<const T*>(p.v_new) + in_off);
+            }
             *reinterpret_cast<uint4*>(static_cast<T*>(p.kc_w) + c_off) = kn;
             *reinterpret_cast<uint4*>(static_cast<T*>(p.vc_w) + c_off) = vsub;
 #pragma unroll
@@ -641,9 +691,13 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
         for (int k = 0; k < NV; ++k) vu[k] = *reinterpret_cast<const uint4*>(Vs + (k * RPI + grp) * RB + sub * 16);
 #pragma unroll
         for (int k = 0; k < NV; ++k) pk[k] = __shfl_sync(0xffffffffu, pr, grp * LPR + k);
+        if (APPEND && sub_k >= 0) {
+#pragma unroll
+          for (int k = 0; k < NV; ++k)
+            if (k == sub_k) vu[k] = vsub;
+        }
 #pragma unroll
         for (int k = 0; k < NV; ++k) {
-          if (APPEND && k == sub_k) vu[k] = vsub;
           if (k * RPI + grp < nr) {
             float f[EPV];
             Vec16<T>::unpack(vu[k], f);

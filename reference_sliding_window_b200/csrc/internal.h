@@ -73,6 +73,10 @@ struct DecodeItem {
 // copy 0.  A decode grid never exceeds kStepSlots CTAs.
 constexpr int kStepSlots = 256;
 
+// Slabs (b, h) the cluster plan serves at most (its per-slab sizes travel in
+// the kernel parameters).
+constexpr int kClusterPlanMaxSlabs = 32;
+
 // Device workspace layout (byte offsets from the workspace base).
 struct WorkspaceLayout {
   size_t err;        // int32: device error word
@@ -118,7 +122,13 @@ struct DecodeParams {
   int ref_stable;        // 1: the reference rows are final (see decode.cu); 0: read after the wait
   int cluster_merge;     // 1: the kDecodeCluster CTAs of a slab form a cluster and merge in
                          //    the leader's shared memory (one item per CTA)
+  int ring_early;        // 1: stages holding ring rows may be copied before the wait too
   float scale_log2;      // softmax scale * log2(e)
+  // Cluster plan: the planned rows and the reference length of each slab
+  // (at most kClusterPlanMaxSlabs), so that a CTA derives its item from its
+  // index with no load from global memory (items/cta_begin then unused).
+  int32_t cl_rows[kClusterPlanMaxSlabs];
+  int32_t cl_lm[kClusterPlanMaxSlabs];
   unsigned long long* timing;  // profiling stamps (RSWA_TIMING builds), may be null
 };
 
