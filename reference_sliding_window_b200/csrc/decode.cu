@@ -170,6 +170,18 @@ __device__ __forceinline__ float fma2_bf16(uint32_t a, uint32_t b, float acc) {
   return acc;
 }
 
+// lo += p2.lo * w.lo, hi += p2.hi * w.hi for packed bf16 pairs, fp32
+// accumulation (P.V with the weight rounded to bf16, as a tensor-core P.V
+// takes it; each product is exact in fp32).
+__device__ __forceinline__ void fma_bf16_pair(uint32_t p2, uint32_t w, float& lo, float& hi) {
+  asm("{.reg .b16 pl, ph, wl, wh;\n\t"
+      "mov.b32 {pl, ph}, %2;\n\t"
+      "mov.b32 {wl, wh}, %3;\n\t"
+      "fma.rn.f32.bf16 %0, pl, wl, %0;\n\t"
+      "fma.rn.f32.bf16 %1, ph, wh, %1;\n\t}"
+      : "+f"(lo), "+f"(hi)
+      : "r"(p2), "r"(w));
+}
 // ---- thread-block cluster helpers (cluster-merge plan)
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
@@ -689,8 +701,18 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
         float pk[NV];
 #pragma unroll
         for (int k = 0; k < NV; ++k) vu[k] = *reinterpret_cast<const uint4*>(Vs + (k * RPI + grp) * RB + sub * 16);
+        // bf16: the weight is rounded once, by the lane that holds it, and
+        // broadcast packed
+        uint32_t pk2[NV];
+        if (kMixed) {
+          uint32_t pr2;
+          asm("cvt.rn.bf16x2.f32 %0, %1, %1;" : "=r"(pr2) : "f"(pr));
 #pragma unroll
-        for (int k = 0; k < NV; ++k) pk[k] = __shfl_sync(0xffffffffu, pr, grp * LPR + k);
+          for (int k = 0; k < NV; ++k) pk2[k] = __shfl_sync(0xffffffffu, pr2, grp * LPR + k);
+        } else {
+#pragma unroll
+          for (int k = 0; k < NV; ++k) pk[k] = __shfl_sync(0xffffffffu, pr, grp * LPR + k);
+        }
         if (APPEND && sub_k >= 0) {
 #pragma unroll
           for (int k = 0; k < NV; ++k)
@@ -699,10 +721,17 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
 #pragma unroll
         for (int k = 0; k < NV; ++k) {
           if (k * RPI + grp < nr) {
-            float f[EPV];
-            Vec16<T>::unpack(vu[k], f);
+            if (kMixed) {
+              fma_bf16_pair(pk2[k], vu[k].x, of[0], of[1]);
+              fma_bf16_pair(pk2[k], vu[k].y, of[2], of[3]);
+              fma_bf16_pair(pk2[k], vu[k].z, of[4], of[5]);
+              fma_bf16_pair(pk2[k], vu[k].w, of[6], of[7]);
+            } else {
+              float f[EPV];
+              Vec16<T>::unpack(vu[k], f);
 #pragma unroll
-            for (int e = 0; e < EPV; ++e) of[e] = fmaf(pk[k], f[e], of[e]);
+              for (int e = 0; e < EPV; ++e) of[e] = fmaf(pk[k], f[e], of[e]);
+            }
           }
         }
       }
@@ -830,34 +859,37 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
       store_elem(static_cast<T*>(p.o) + (size_t)item.bh * D + tid, acc / L);
     }
   }
-  // ---- split items: the CTA holding the last ticket of a slab merges it.
-  if (tid == 0) {
-    int l0 = 0, l1 = 0;
-    if (pend0 >= 0) l0 = tk0 == item_at(pend0).nparts - 1;
-    if (pend1 >= 0) l1 = tk1 == item_at(pend1).nparts - 1;
-    if (l0 || l1) fence_acq_rel_gpu();  // acquire the other CTAs' partials
-    s_flag[0] = l0;
-    s_flag[1] = l1;
-    RSWA_STAMP(11);
-  }
-  named_barrier_sync(1, NT);
-  {
-    // the slabs this CTA merges (uniform across the CTA): m0, then m1
-    const int f0 = s_flag[0], f1 = s_flag[1];
-    const int nm = f0 + f1;
-    if (nm > 0) {
-      const DecodeItem m0 = item_at(f0 ? pend0 : pend1);
-      const DecodeItem m1 = item_at(pend1 >= 0 ? pend1 : pend0);
-      // The host planner keeps every slab within kMergeCap / 2 partials.
-      if (m0.nparts + (nm > 1 ? m1.nparts : 0) <= Tr::kMergeCap) {
-        merge_partials_joint<T, D, NT>(p, m0, m1, nm, tid, merge_buf);
-      } else if (tid == 0) {
-        flag_error(p.err, kErrPlanShort);
-      }
-      if (tid == 0) {
-        RSWA_STAMP(13);
-        p.tickets[m0.bh] = 0;
-        if (nm > 1) p.tickets[m1.bh] = 0;
+  // ---- split items (span plan): the CTA holding the last ticket of a slab
+  // merges it.  (The condition is uniform across the CTA.)
+  if (!p.cluster_merge) {
+    if (tid == 0) {
+      int l0 = 0, l1 = 0;
+      if (pend0 >= 0) l0 = tk0 == item_at(pend0).nparts - 1;
+      if (pend1 >= 0) l1 = tk1 == item_at(pend1).nparts - 1;
+      if (l0 || l1) fence_acq_rel_gpu();  // acquire the other CTAs' partials
+      s_flag[0] = l0;
+      s_flag[1] = l1;
+      RSWA_STAMP(11);
+    }
+    named_barrier_sync(1, NT);
+    {
+      // the slabs this CTA merges (uniform across the CTA): m0, then m1
+      const int f0 = s_flag[0], f1 = s_flag[1];
+      const int nm = f0 + f1;
+      if (nm > 0) {
+        const DecodeItem m0 = item_at(f0 ? pend0 : pend1);
+        const DecodeItem m1 = item_at(pend1 >= 0 ? pend1 : pend0);
+        // The host planner keeps every slab within kMergeCap / 2 partials.
+        if (m0.nparts + (nm > 1 ? m1.nparts : 0) <= Tr::kMergeCap) {
+          merge_partials_joint<T, D, NT>(p, m0, m1, nm, tid, merge_buf);
+        } else if (tid == 0) {
+          flag_error(p.err, kErrPlanShort);
+        }
+        if (tid == 0) {
+          RSWA_STAMP(13);
+          p.tickets[m0.bh] = 0;
+          if (nm > 1) p.tickets[m1.bh] = 0;
+        }
       }
     }
   }
