@@ -546,9 +546,16 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
    for (int x = 0; x < nb; ++x) {
     const int it = it0 + x;
     const int li = it - it_begin;
-    const DecodeItem item = li < kPreItems ? s_items[li] : p.items[it];
-    const int b = item.bh / p.H;
-    const int Lm_b = li < kPreItems ? s_lm[li] : p.Lm[b];
+    // (branches, not selects: the staged case must not wait on a global load)
+    DecodeItem item;
+    int Lm_b;
+    if (li < kPreItems) {
+      item = s_items[li];
+      Lm_b = s_lm[li];
+    } else {
+      item = p.items[it];
+      Lm_b = p.Lm[item.bh / p.H];
+    }
     const int T_now = T_step;
     const int len = valid_rows(p, Lm_b, T_now);
     const int live = max(0, min(len - item.row0, item.rows));  // rows to attend
@@ -568,8 +575,10 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
     float qf[EPV], of[EPV];
     uint4 qraw = make_uint4(0, 0, 0, 0);
     if (kMixed) {
-      qraw = li < kPreItems ? reinterpret_cast<const uint4*>(s_q + li * D)[sub]
-                            : *reinterpret_cast<const uint4*>(static_cast<const T*>(p.q) + (size_t)item.bh * D + sub * EPV);
+      if (li < kPreItems)
+        qraw = reinterpret_cast<const uint4*>(s_q + li * D)[sub];
+      else
+        qraw = *reinterpret_cast<const uint4*>(static_cast<const T*>(p.q) + (size_t)item.bh * D + sub * EPV);
     } else if (li < kPreItems) {
 #pragma unroll
       for (int e = 0; e < EPV; e += 4) {
