@@ -15,8 +15,10 @@ step is constant; exactly K steps are timed.
 
 value     : tokens/s through one attention layer = B * R * K / device time.
 e2e       : the same through the public binding with HOST buffers: every step
-            copies q, k, v of all R layers from pinned host memory, runs the R
-            calls and copies the outputs back, all inside the timed region.
+            copies q, k, v of all R layers from pinned host memory, runs the
+            step (a LayerStep built once with graph=True: one CUDA graph of the
+            R launches) and copies the outputs back, all inside the timed
+            region.
 roofline  : algorithmic bytes per launch (2 * rows * d * 2 bytes of K and V
             plus q, o, new k, v) / average launch time, against the measured
             HBM copy bandwidth.
@@ -543,7 +545,7 @@ def run_decode(args, name, w, lens, T_target, steps, warmup, e2e_steps):
     # the step over the staging buffers, made once (as a model holds its buffers)
     with torch.cuda.stream(stream):
         step_e2e = LayerStep(layers, [dev_in[r, 0] for r in range(R)], [dev_in[r, 1] for r in range(R)],
-                             [dev_in[r, 2] for r in range(R)], outs)
+                             [dev_in[r, 2] for r in range(R)], outs, graph=True)
         torch.cuda.synchronize(dev)
         e0.record(stream)
         for i in range(K_e2e):

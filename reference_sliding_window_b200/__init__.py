@@ -273,10 +273,18 @@ class LayerStep:
     """One decode step over fixed layer handles and fixed device buffers (a
     model's per-layer k, v, q and output tensors, refilled in place every
     step): the checks and the pointer arrays are done once, so each call is
-    a single C call of rswa_append_decode_layers."""
+    a single C call of rswa_append_decode_layers.
+
+    graph=True (RSWA-mode handles only) captures that call once into a CUDA
+    graph and replays it on each call: the step counter lives on the device,
+    so every replay is the next step.  Capture and replays do not keep the
+    handles' host-side step count (read only by FULL-mode planning and the
+    reference-chunk loader); step_count() reads the device counter and
+    refreshes it."""
 
     def __init__(self, layers: Sequence[RSWA], k: Sequence[torch.Tensor], v: Sequence[torch.Tensor],
-                 q: Sequence[torch.Tensor], out: Sequence[torch.Tensor], scale: float = 0.0):
+                 q: Sequence[torch.Tensor], out: Sequence[torch.Tensor], scale: float = 0.0,
+                 graph: bool = False):
         R = len(layers)
         if not (len(k) == len(v) == len(q) == len(out) == R) or R < 1:
             raise ValueError("one k, v, q and out per layer")
@@ -292,11 +300,30 @@ class LayerStep:
                       P(*[t.data_ptr() for t in v]), P(*[t.data_ptr() for t in q]),
                       P(*[t.data_ptr() for t in out]), float(scale))
         self._fn = _native.lib().rswa_append_decode_layers
+        self._graph = None
+        if graph:
+            if any(a.mode != MODE_RSWA for a in layers):
+                raise ValueError("graph=True needs RSWA-mode handles (FULL mode re-plans on the host)")
+            dev = layers[0].device
+            side = torch.cuda.Stream(dev)
+            side.wait_stream(torch.cuda.current_stream(dev))
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(side):
+                with torch.cuda.graph(g, stream=side):
+                    self._launch()
+            torch.cuda.current_stream(dev).wait_stream(side)
+            self._graph = g
 
-    def __call__(self) -> None:
+    def _launch(self) -> None:
         for a in self._layers:
             a._sync_stream()
         check(self._fn(*self._args))
+
+    def __call__(self) -> None:
+        if self._graph is not None:
+            self._graph.replay()
+        else:
+            self._launch()
 
 
 def masked_forward(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, L_m: int, n: int,

@@ -77,7 +77,7 @@ def test_reference_in_chunks_equals_one_load(dtype, d):
     a.check()
 
 
-@pytest.mark.parametrize("graph", [False, True, "step"])
+@pytest.mark.parametrize("graph", [False, True, "step", "graphstep"])
 def test_layers_call_every_layer_matches_the_oracle(graph):
     """R = 4 layers of different reference lengths and the same batch; the
     queries spike on window edges at the sampled steps."""
@@ -92,11 +92,11 @@ def test_layers_call_every_layer_matches_the_oracle(graph):
     ins = [tuple(t.to(dev) for t in (c.k, c.v, c.q)) for c in cases]
     outs = [torch.empty_like(ins[r][2][0]) for r in range(R)]
     got = {r: {} for r in range(R)}
-    if graph == "step":  # fixed buffers refilled in place, one prebuilt C call per step
+    if graph in ("step", "graphstep"):  # fixed buffers refilled in place, one prebuilt call per step
         kin = [x[0][0].clone() for x in ins]
         vin = [x[1][0].clone() for x in ins]
         qin = [x[2][0].clone() for x in ins]
-        step = LayerStep(layers, kin, vin, qin, outs)
+        step = LayerStep(layers, kin, vin, qin, outs, graph=graph == "graphstep")
         for t in range(1, T + 1):
             for r in range(R):
                 kin[r].copy_(ins[r][0][t - 1])
