@@ -282,7 +282,9 @@ __device__ __forceinline__ void merge_partials_joint(const DecodeParams& p, cons
   named_barrier_sync(1, NT);
 }
 
-template <typename T, int D, bool APPEND>
+// CLUSTER: the cluster plan (a separate instantiation, so that neither plan
+// carries the other's code and registers).
+template <typename T, int D, bool APPEND, bool CLUSTER>
 __global__ void __launch_bounds__(DecTraits<T, D>::kThreads, 1)
 decode_kernel(const __grid_constant__ DecodeParams p) {
   using Tr = DecTraits<T, D>;
@@ -323,7 +325,7 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
       mbar_init(smem_u32(&empty_bar[s]), 32 * Tr::kSplit);  // every lane of the owning group
     }
     *s_abort = 0;
-    if (p.cluster_merge) mbar_init(cl_bar, 1);  // the leader's own arrival; the others complete bytes
+    if (CLUSTER) mbar_init(cl_bar, 1);  // the leader's own arrival; the others complete bytes
     fence_barrier_init();
   }
   // The plan and the reference lengths are written by host copies ordered
@@ -335,13 +337,13 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
   // Cluster plan: one item per CTA, derived from the CTA index and the
   // per-slab sizes in the parameters exactly as the host planner makes it,
   // so no chain of dependent global loads delays the first copies.
-  const int it_begin = p.cluster_merge ? (int)blockIdx.x : p.cta_begin[blockIdx.x];
-  const int it_end = p.cluster_merge ? (int)blockIdx.x + 1 : p.cta_begin[blockIdx.x + 1];
+  const int it_begin = CLUSTER ? (int)blockIdx.x : p.cta_begin[blockIdx.x];
+  const int it_end = CLUSTER ? (int)blockIdx.x + 1 : p.cta_begin[blockIdx.x + 1];
   const int n_pre = min(it_end - it_begin, kPreItems);
   if ((int)threadIdx.x < n_pre) {
     DecodeItem item;
     int lm;
-    if (p.cluster_merge) {
+    if (CLUSTER) {
       const int c = blockIdx.x, bh = c / kDecodeCluster, r = c % kDecodeCluster;
       const int rows_bh = p.cl_rows[bh], S = (rows_bh + 31) / 32;
       const int st0 = (int)((long long)S * r / kDecodeCluster), st1 = (int)((long long)S * (r + 1) / kDecodeCluster);
@@ -365,7 +367,7 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
   // Cluster-merge plan: the leader's barrier must be initialised before any
   // CTA of the cluster arrives on it.  Every thread passes here (no thread
   // has exited yet), so this hardware barrier cannot be left waiting.
-  if (p.cluster_merge) cluster_sync_all();
+  if (CLUSTER) cluster_sync_all();
   auto item_at = [&](int it) -> DecodeItem {
     const int li = it - it_begin;
     return li < kPreItems ? s_items[li] : p.items[it];
@@ -788,7 +790,7 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
       }
       if (item.nparts == 1) {
         store_elem(static_cast<T*>(p.o) + (size_t)item.bh * D + dd, acc / Ls);
-      } else if (p.cluster_merge) {
+      } else if (CLUSTER) {
         // this CTA's partial into slot `rank` of the cluster leader's buffer
         float* mine = cl_buf + (size_t)cluster_rank() * (D + 4);
         mine[dd] = acc;
@@ -808,7 +810,7 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
     }
     named_barrier_sync(1, NT);  // partials written; red_* are reused by the next batch
     if (tid == 0 && it0 == it_begin) RSWA_STAMP(10);
-    if (p.cluster_merge) {
+    if (CLUSTER) {
       // one item per CTA: arrive on the leader's barrier with release at
       // cluster scope (after the barrier, so it covers every thread's stores)
       if (tid == 0 && item_at(it0).nparts > 1) {
@@ -850,7 +852,7 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
 
   if (tid == 0) RSWA_STAMP(4);
   // ---- cluster-merge plan: the leader folds the cluster's partials
-  if (p.cluster_merge && it_end > it_begin && cluster_rank() == 0 && item_at(it_begin).nparts > 1 && tid < D) {
+  if (CLUSTER && it_end > it_begin && cluster_rank() == 0 && item_at(it_begin).nparts > 1 && tid < D) {
     const DecodeItem item = item_at(it_begin);
     const bool ok = mbar_wait_cluster_bounded(cl_bar, 0);
     if (!ok && tid == 0) flag_error(p.err, kErrWaitTimeout);
@@ -870,7 +872,7 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
   }
   // ---- split items (span plan): the CTA holding the last ticket of a slab
   // merges it.  (The condition is uniform across the CTA.)
-  if (!p.cluster_merge) {
+  if (!CLUSTER) {
     if (tid == 0) {
       int l0 = 0, l1 = 0;
       if (pend0 >= 0) l0 = tk0 == item_at(pend0).nparts - 1;
@@ -904,7 +906,7 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
   }
 
   if (tid == 0) RSWA_STAMP(5);
-  if (p.cluster_merge && tid == 0) bulk_wait_read();  // the partial has left this CTA's shared memory
+  if (CLUSTER && tid == 0) bulk_wait_read();  // the partial has left this CTA's shared memory
   // Advance T: copies blockIdx.x, blockIdx.x + grid, ... (kStepSlots <= NT,
   // one store per thread), none of which another CTA of this launch reads.
   if (APPEND && !(p.full_mode && T0 + 1 > p.T_cap)) {
@@ -920,7 +922,10 @@ static cudaError_t launch_one(const DecodeParams& p, int grid, cudaStream_t stre
   using Tr = DecTraits<T, D>;
   static PerContextOnce attr_once;
   cudaError_t e = attr_once.run([] {
-    return cudaFuncSetAttribute(decode_kernel<T, D, A>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e1 = cudaFuncSetAttribute(decode_kernel<T, D, A, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)Tr::kSmemBytes);
+    if (e1 != cudaSuccess) return e1;
+    return cudaFuncSetAttribute(decode_kernel<T, D, A, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)Tr::kSmemBytes);
   });
   if (e != cudaSuccess) return e;
@@ -938,13 +943,14 @@ static cudaError_t launch_one(const DecodeParams& p, int grid, cudaStream_t stre
   attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = p.cluster_merge ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, decode_kernel<T, D, A>, p);
+  return p.cluster_merge ? cudaLaunchKernelEx(&cfg, decode_kernel<T, D, A, true>, p)
+                         : cudaLaunchKernelEx(&cfg, decode_kernel<T, D, A, false>, p);
 }
 
 template <typename T, int D>
 static int max_clusters(void) {
   using Tr = DecTraits<T, D>;
-  if (cudaFuncSetAttribute(decode_kernel<T, D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(decode_kernel<T, D, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)Tr::kSmemBytes) != cudaSuccess)
     return 0;
   cudaLaunchConfig_t cfg = {};
@@ -959,7 +965,7 @@ static int max_clusters(void) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, decode_kernel<T, D, true>, &cfg) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&n, decode_kernel<T, D, true, true>, &cfg) != cudaSuccess) {
     cudaGetLastError();  // clear the sticky-free error so later calls are unaffected
     return 0;
   }
