@@ -638,6 +638,7 @@ static rswa_status run_decode(rswa_ctx* c, const void* k, const void* v, const v
   p.H = c->H;
   p.S_cap = c->S_cap;
   p.n = c->n;
+  set_mod_magic(p, c->n);
   p.full_mode = c->mode == RSWA_MODE_FULL;
   p.T_cap = c->T_cap;
   p.n_ctas = c->n_ctas;

@@ -231,6 +231,16 @@ __device__ __forceinline__ void griddep_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// x mod n for 0 <= x < 2^31 by a multiply (the divisor's magic number comes
+// with the parameters): q = floor(x * M / 2^k) with k = 32 + ceil(log2 n)
+// and M = ceil(2^k / n) is exact there, since M * n - 2^k < n <= 2^(k-32)
+// keeps the error of x * M / 2^k below 1 / n (Granlund and Montgomery,
+// "Division by invariant integers using multiplication", 1994).
+__device__ __forceinline__ int mod_n(const DecodeParams& p, int x) {
+  const unsigned q = (unsigned)(((unsigned long long)(unsigned)x * p.n_magic) >> p.n_shift);
+  return x - (int)q * p.n;
+}
+
 // Valid cache rows of a sequence with Lm reference rows when the step
 // counter reads T_now.
 __device__ __forceinline__ int valid_rows(const DecodeParams& p, int Lm, int T_now) {
@@ -570,7 +580,7 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
         if (T_now <= p.T_cap) slot_row = Lm_b + T_now - 1;
         else if (tid == 0 && item.row0 == 0) flag_error(p.err, kErrCapacity);
       } else {
-        slot_row = Lm_b + (T_now - 1) % p.n;
+        slot_row = Lm_b + mod_n(p, T_now - 1);
       }
     }
 

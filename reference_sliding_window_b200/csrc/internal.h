@@ -108,6 +108,8 @@ struct DecodeParams {
   const void* v_new;
   int B, H, S_cap;
   int n;                 // ring size (RSWA mode)
+  int n_shift;           // x mod n = x - n * ((x * n_magic) >> n_shift) for 0 <= x < 2^31
+  unsigned long long n_magic;
   int full_mode;         // 0: ring of n slots, 1: outputs in order
   int T_cap;             // FULL mode capacity
   int n_ctas;            // grid size; CTA c runs items [cta_begin[c], cta_begin[c+1])
@@ -131,6 +133,14 @@ struct DecodeParams {
   int32_t cl_lm[kClusterPlanMaxSlabs];
   unsigned long long* timing;  // profiling stamps (RSWA_TIMING builds), may be null
 };
+
+// The decode kernel's magic number for x mod n (mod_n in decode.cu).
+inline void set_mod_magic(DecodeParams& p, int n) {
+  int s = 0;
+  while ((1LL << s) < (long long)n) ++s;
+  p.n_shift = 32 + s;
+  p.n_magic = ((1ULL << p.n_shift) + (unsigned long long)n - 1) / (unsigned long long)n;
+}
 
 // Launch the split-K decode kernel (append: fused ring write + T advance).
 // CTAs per cluster in the cluster-merge plan.

@@ -180,6 +180,7 @@ extern "C" rswa_status rswa_decode_noalloc(const void* k_cache, const void* v_ca
   p.H = H;
   p.S_cap = S_cap;
   p.n = 1;
+  set_mod_magic(p, 1);
   p.full_mode = 1;  // with T = 0 the attended rows are exactly cache_lens[b]
   p.T_cap = 0;
   p.n_ctas = G;
