@@ -185,7 +185,7 @@ static void make_plan(rswa_ctx* c) {
       const int S = stages[bh];
       for (int r = 0; r < kDecodeCluster; ++r) {
         const int g = bh * kDecodeCluster + r;
-        const int st0 = (int)((long long)S * r / kDecodeCluster), st1 = (int)((long long)S * (r + 1) / kDecodeCluster);
+        const int st0 = cluster_stage_begin(S, r), st1 = cluster_stage_begin(S, r + 1);
         DecodeItem it{};
         it.bh = bh;
         it.row0 = st0 * 32;

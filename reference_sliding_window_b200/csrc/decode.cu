@@ -356,7 +356,7 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
     if (CLUSTER) {
       const int c = blockIdx.x, bh = c / kDecodeCluster, r = c % kDecodeCluster;
       const int rows_bh = p.cl_rows[bh], S = (rows_bh + 31) / 32;
-      const int st0 = (int)((long long)S * r / kDecodeCluster), st1 = (int)((long long)S * (r + 1) / kDecodeCluster);
+      const int st0 = cluster_stage_begin(S, r), st1 = cluster_stage_begin(S, r + 1);
       item.bh = bh;
       item.row0 = st0 * 32;
       item.rows = max(0, min(rows_bh, st1 * 32) - item.row0);

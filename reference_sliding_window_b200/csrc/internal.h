@@ -145,6 +145,18 @@ inline void set_mod_magic(DecodeParams& p, int n) {
 // Launch the split-K decode kernel (append: fused ring write + T advance).
 // CTAs per cluster in the cluster-merge plan.
 constexpr int kDecodeCluster = 8;
+// First 32-row stage of cluster rank r's share of a slab with S stages.
+// With at least one stage per rank: S / 8 stages each, and the S mod 8
+// extra ones to ranks 1, 2, ... (the leader merges the cluster and the last
+// rank holds the ring, so both get the short shares when they can).  Fewer
+// stages than ranks: floor(S * r / 8), so the last rank still ends the slab.
+__host__ __device__ inline int cluster_stage_begin(int S, int r) {
+  if (r >= kDecodeCluster) return S;
+  if (S < kDecodeCluster) return (int)((long long)S * r / kDecodeCluster);
+  const int q = S / kDecodeCluster, rem = S % kDecodeCluster;
+  const int extra = r <= 0 ? 0 : (r - 1 < rem ? r - 1 : rem);
+  return r * q + extra;
+}
 // Clusters of kDecodeCluster decode CTAs that can be resident at once (0 on error).
 int decode_max_active_clusters(int elem, int D);
 
