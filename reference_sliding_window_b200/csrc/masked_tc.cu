@@ -561,16 +561,16 @@ __global__ void __launch_bounds__(kThreads, 1) masked_tc_kernel(const __grid_con
           we = i - k0;
         }
       }
-      // pass 1: row maximum over the 128 scores
-      float mh = -INFINITY;
-#pragma unroll 1
-      for (int c0 = 0; c0 < kTile; c0 += kHalf) {
-        float s[kHalf];
-        tmem_ld32(lane_base + colS + c0, s);
-        tmem_ld32(lane_base + colS + c0 + 32, s + 32);
-        tmem_wait_ld();
-        mh = fmaxf(mh, full ? half_max<true>(s, c0, ra, wb, we) : half_max<false>(s, c0, ra, wb, we));
-      }
+      // the 128 scores into registers once: pass 1 (maximum) and pass 2
+      // (exponentials) read them there
+      float s[kTile];
+      tmem_ld32(lane_base + colS, s);
+      tmem_ld32(lane_base + colS + 32, s + 32);
+      tmem_ld32(lane_base + colS + 64, s + 64);
+      tmem_ld32(lane_base + colS + 96, s + 96);
+      tmem_wait_ld();
+      const float mh = full ? fmaxf(half_max<true>(s, 0, ra, wb, we), half_max<true>(s + kHalf, kHalf, ra, wb, we))
+                            : fmaxf(half_max<false>(s, 0, ra, wb, we), half_max<false>(s + kHalf, kHalf, ra, wb, we));
       if (stamp) TC_CYC(j, 2);
       // lazy rescale: only when the max (log2 units) grew by more than 8
       const float mt_s = mh * p.scale_log2;
@@ -578,18 +578,13 @@ __global__ void __launch_bounds__(kThreads, 1) masked_tc_kernel(const __grid_con
       const float m_new = grow ? mt_s : m_ref;
       const float corr = grow ? ex2(m_ref - m_new) : 1.f;  // 0 when m_ref was -inf
       const float msub = (m_new == -INFINITY) ? 0.f : m_new;
-      // pass 2: exponentials; P (bf16 pairs) goes over S columns [0, 64),
-      // which pass 2 has read by the time it writes them
+      // pass 2: exponentials; P (bf16 pairs) goes over S columns [0, 64)
       float lt = 0.f;
-#pragma unroll 1
+#pragma unroll
       for (int c0 = 0; c0 < kTile; c0 += kHalf) {
-        float s[kHalf];
-        tmem_ld32(lane_base + colS + c0, s);
-        tmem_ld32(lane_base + colS + c0 + 32, s + 32);
-        tmem_wait_ld();
         uint32_t pk[kHalf / 2];
-        lt += full ? half_exp<true>(s, c0, ra, wb, we, p.scale_log2, msub, pk)
-                   : half_exp<false>(s, c0, ra, wb, we, p.scale_log2, msub, pk);
+        lt += full ? half_exp<true>(s + c0, c0, ra, wb, we, p.scale_log2, msub, pk)
+                   : half_exp<false>(s + c0, c0, ra, wb, we, p.scale_log2, msub, pk);
         tmem_st_pairs(lane_base + colS + c0 / 2, pk);
       }
       if (stamp) TC_CYC(j, 3);
