@@ -395,15 +395,15 @@ extern "C" rswa_status rswa_init(rswa_handle* out, rswa_mode mode, int L_m_cap, 
 static std::mutex g_last_decode_mu;
 static std::map<std::pair<int, cudaStream_t>, const rswa_ctx*> g_last_decode;
 
+// The caller holds g_last_decode_mu from the query until its launch is
+// enqueued and noted, so the record follows the stream's launch order even
+// when host threads share a stream; a launch that fails is not noted.
 static bool previous_decode_is(const rswa_ctx* c) {
   if (c->stream == cudaStreamPerThread) return true;
-  std::lock_guard<std::mutex> lock(g_last_decode_mu);
-  const auto key = std::make_pair(c->device, c->stream);
-  auto it = g_last_decode.find(key);
-  const bool same = it != g_last_decode.end() && it->second == c;
-  g_last_decode[key] = c;
-  return same;
+  auto it = g_last_decode.find(std::make_pair(c->device, c->stream));
+  return it != g_last_decode.end() && it->second == c;
 }
+static void note_decode(const rswa_ctx* c) { g_last_decode[std::make_pair(c->device, c->stream)] = c; }
 
 extern "C" void rswa_destroy(rswa_handle h) {
   if (!h) return;
@@ -662,7 +662,6 @@ static rswa_status run_decode(rswa_ctx* c, const void* k, const void* v, const v
   p.ring_early = 0;
 #else
   p.ref_stable = 1;
-  p.ring_early = previous_decode_is(c) ? 0 : 1;
 #endif
   if (c->cluster_plan)
     for (int bh = 0; bh < c->B * c->H; ++bh) {
@@ -670,8 +669,15 @@ static rswa_status run_decode(rswa_ctx* c, const void* k, const void* v, const v
       p.cl_lm[bh] = c->cl_lm[bh];
     }
   const int grid = c->n_ctas;
-  RSWA_CUDA(launch_decode(c->dtype == RSWA_BF16 ? kBF16 : kF32, c->d, append, p, grid, c->stream),
-            "decode kernel");
+  {
+    std::lock_guard<std::mutex> lock(g_last_decode_mu);  // record and launch in one order
+#ifndef RSWA_NO_EARLY_COPY
+    p.ring_early = previous_decode_is(c) ? 0 : 1;
+#endif
+    RSWA_CUDA(launch_decode(c->dtype == RSWA_BF16 ? kBF16 : kF32, c->d, append, p, grid, c->stream),
+              "decode kernel");
+    if (c->stream != cudaStreamPerThread) note_decode(c);
+  }
   if (append) c->T_host += 1;
   return RSWA_OK;
 }
