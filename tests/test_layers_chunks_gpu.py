@@ -77,16 +77,21 @@ def test_reference_in_chunks_equals_one_load(dtype, d):
     a.check()
 
 
-@pytest.mark.parametrize("graph", [False, True, "step", "graphstep"])
-def test_layers_call_every_layer_matches_the_oracle(graph):
-    """R = 4 layers of different reference lengths and the same batch; the
-    queries spike on window edges at the sampled steps."""
-    R, T, n = 4, 150, 16
+@pytest.mark.parametrize("graph,R", [(False, 4), (True, 4), ("step", 4), ("graphstep", 4), ("graphstep", 2)])
+def test_layers_call_every_layer_matches_the_oracle(graph, R):
+    """R layers of different reference lengths and the same batch; the
+    queries spike on window edges at the sampled steps.  With R = 2 each
+    decode's previous kernel is the other layer's, the tightest case for
+    copying ring rows before the dependency wait."""
+    T, n = 150, 16
     cases = [synth.decode_case(B=2, H=2, d=128, ref_lens=[300 + 37 * r, 41 + r], n=n, T=T, dtype="bf16",
                                seed=70 + r) for r in range(R)]
-    steps = {1, n, n + 1, 2 * n + 1, T}
+    edge_steps = {1, n, n + 1, 2 * n + 1, T}
+    prev_steps = {n + 5, T - 1}  # queries on the output the previous step appended
+    steps = edge_steps | prev_steps
     for c in cases:
-        synth.spike_decode_queries(c, spikes.decode_edge_probes(sorted(steps), c.ref_lens, n))
+        synth.spike_decode_queries(c, spikes.decode_edge_probes(sorted(edge_steps), c.ref_lens, n))
+        synth.spike_decode_queries(c, [(t, b, c.ref_lens[b] + t - 1) for t in sorted(prev_steps) for b in range(c.B)])
     layers = [make_attn(c) for c in cases]
     dev = layers[0].device
     ins = [tuple(t.to(dev) for t in (c.k, c.v, c.q)) for c in cases]
