@@ -1,10 +1,12 @@
 """GPU tests of consecutive decode launches on one handle with nothing in
 between, captured in one CUDA graph, so each launch may start (and copy
-cache rows) while the previous step is still running.  The decode copies
-ring rows before its dependency wait; the one row such a copy can miss, the
-slot of the token the previous launch appended, is taken from the side copy
-that launch leaves.  Every step is checked against the oracle, with queries
-spiked on the newest outputs so a stale row fails by O(1).
+reference rows) while the previous step is still running.  The library
+then copies ring rows only after the dependency wait: the previous kernel
+on the stream is a decode of the same handle, which may still be writing
+its slot row.  Every step is checked against the oracle, with queries
+spiked on the output the previous step appended, so a stale copy of that
+row fails by O(1).  Also after a packed load and after a reset, and in
+FULL mode.
 
 Spec: "Unlimited OCR Works", 方法展开 §3-§4 (Eq.(3)-(4) over the Eq.(6)
 cache; output T overwrites the slot of output T - n).
