@@ -13,7 +13,7 @@
 // The caller passes the caches, the query and the output.  Every call reuses
 // the same array, so two calls whose kernels overlap on the GPU race; issue
 // them on one stream (or otherwise order them).  The parts that must start at
-// zero (launch ticket, step counter, split-K tickets) are cleared by every
+// zero (step counter, split-K tickets) are cleared by every
 // call; the device error word is kept until rswa_decode_noalloc_check reads
 // and clears it.
 
@@ -37,7 +37,7 @@ constexpr int kNoAllocMaxD = 128;
 
 // Scratch layout (bytes), every region 256-byte aligned.
 constexpr size_t kNaErr = 0;                                       // int32 error word
-constexpr size_t kNaDone = 4;                                      // int32 launch ticket
+constexpr size_t kNaDone = 4;                                      // unused (zeroed with the counter)
 constexpr size_t kNaT = 256;                                       // int32 step counter (always 0)
 constexpr size_t kNaLm = 512;                                      // int32[max slabs]
 constexpr size_t kNaTickets = kNaLm + 4 * kNoAllocMaxSlabs;        // int32[max slabs]
