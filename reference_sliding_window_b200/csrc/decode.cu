@@ -16,7 +16,9 @@
 //   items at slab boundaries, so only the first and last item of a CTA can
 //   be part of a slab shared with another CTA.  Cluster plan, when every
 //   slab can have a resident cluster of its own: slab bh goes to the
-//   kDecodeCluster CTAs of cluster bh, one contiguous part each.
+//   kDecodeCluster CTAs of cluster bh, one contiguous part each (the leader
+//   and the last rank take the short shares).  Each plan is its own kernel
+//   instantiation (template parameter CLUSTER).
 // * Before waiting on the previous kernel (programmatic dependent launch):
 //   barrier set-up, the plan and reference lengths (host-written) staged in
 //   shared memory, copies of the leading stages (reference rows, and ring
@@ -38,9 +40,10 @@
 //   mixed-precision FMAs on the packed words) and reduces them with a
 //   transposed butterfly over NV lanes plus plain shuffles over the rest of
 //   the row's lanes (NV-1 + log2(LPR/NV) shuffles leave every lane one
-//   finished score), then updates a float32 online softmax (base 2) and its
-//   slice of the output.  Rows at or past the current cache length are
-//   masked.  Splitting stages over warps keeps the serial work of one warp
+//   finished score), then updates a float32 online softmax (base 2, with a
+//   lazy running maximum) and its slice of the output (bf16 caches: P.V with
+//   the weight rounded to bf16, fp32 accumulation).  Rows at or past the
+//   current cache length are masked.  Splitting stages over warps keeps the serial work of one warp
 //   short (at small cache sizes the launch is latency-bound) while the
 //   copies stay 8 KB each.
 // * Warps merge per batch of items in shared memory.  Items of a shared
