@@ -297,6 +297,25 @@ __device__ __forceinline__ void merge_partials_joint(const DecodeParams& p, cons
 
 // CLUSTER: the cluster plan (a separate instantiation, so that neither plan
 // carries the other's code and registers).
+// The fused append's slot row (taken by one lane group of one part per
+// slab and step), kept out of line so the part's code stays compact.
+template <typename T, int D>
+__device__ __noinline__ void slot_row_kv(const DecodeParams& p, int bh, int slot_row, int li, int sub,
+                                         const uint8_t* s_kn, const uint8_t* s_vn, uint4& kn, uint4& vn) {
+  constexpr int EPV = 16 / (int)sizeof(T), RB = D * (int)sizeof(T);
+  const size_t in_off = (size_t)bh * D + sub * EPV;
+  const size_t c_off = ((size_t)bh * p.S_cap + slot_row) * D + sub * EPV;
+  if (li < kPreItems) {
+    kn = reinterpret_cast<const uint4*>(s_kn + li * RB)[sub];
+    vn = reinterpret_cast<const uint4*>(s_vn + li * RB)[sub];
+  } else {
+    kn = *reinterpret_cast<const uint4*>(static_cast<const T*>(p.k_new) + in_off);
+    vn = *reinterpret_cast<const uint4*>(static_cast<const T*>(p.v_new) + in_off);
+  }
+  *reinterpret_cast<uint4*>(static_cast<T*>(p.kc_w) + c_off) = kn;
+  *reinterpret_cast<uint4*>(static_cast<T*>(p.vc_w) + c_off) = vn;
+}
+
 template <typename T, int D, bool APPEND, bool CLUSTER>
 __global__ void __launch_bounds__(DecTraits<T, D>::kThreads, 1)
 decode_kernel(const __grid_constant__ DecodeParams p) {
@@ -648,18 +667,8 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
           if (rel >= 0 && rel < NV * RPI && rel % RPI == 0) {
             // The new token: use its k/v from the inputs and store it into its slot.
             sub_k = rel / RPI;
-            const size_t in_off = (size_t)item.bh * D + sub * EPV;
-            const size_t c_off = ((size_t)item.bh * p.S_cap + slot_row) * D + sub * EPV;
             uint4 kn;
-            if (li < kPreItems) {
-              kn = reinterpret_cast<const uint4*>(s_kn + li * RB)[sub];
-              vsub = reinterpret_cast<const uint4*>(s_vn + li * RB)[sub];
-            } else {
-              kn = *reinterpret_cast<const uint4*>(static_cast<const T*>(p.k_new) + in_off);
-              vsub = *reinterpret_cast<const uint4*>(static_cast<const T*>(p.v_new) + in_off);
-            }
-            *reinterpret_cast<uint4*>(static_cast<T*>(p.kc_w) + c_off) = kn;
-            *reinterpret_cast<uint4*>(static_cast<T*>(p.vc_w) + c_off) = vsub;
+            slot_row_kv<T, D>(p, item.bh, slot_row, li, sub, s_kn, s_vn, kn, vsub);
 #pragma unroll
             for (int k = 0; k < NV; ++k)
               if (k == sub_k) ku[k] = kn;
