@@ -331,6 +331,35 @@ __device__ __forceinline__ float half_exp(const float* s, int col0, int ra, int 
   return (l4[0] + l4[1]) + (l4[2] + l4[3]);
 }
 
+// half_exp that also returns the maximum of the visible raw scores (for the
+// speculative pass: the exponentials use the maximum in use, and this tile's
+// maximum only decides whether the pass must be redone).
+template <bool FULL>
+__device__ __forceinline__ float half_exp_max(const float* s, int col0, int ra, int wb, int we, float sl2, float msub,
+                                              uint32_t* pk, float& mx) {
+  float l4[4] = {0.f, 0.f, 0.f, 0.f};
+  float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+  for (int e = 0; e < kHalf; e += 2) {
+    const int c = col0 + e;
+    float x0 = fmaf(s[e], sl2, -msub), x1 = fmaf(s[e + 1], sl2, -msub);
+    float s0 = s[e], s1 = s[e + 1];
+    if (!FULL) {
+      const bool v0 = c < ra || (c >= wb && c <= we), v1 = c + 1 < ra || (c + 1 >= wb && c + 1 <= we);
+      x0 = v0 ? x0 : -INFINITY;
+      x1 = v1 ? x1 : -INFINITY;
+      s0 = v0 ? s0 : -INFINITY;
+      s1 = v1 ? s1 : -INFINITY;
+    }
+    m4[(e >> 1) & 3] = max3(m4[(e >> 1) & 3], s0, s1);
+    const float p0 = ex2(x0), p1 = ex2(x1);
+    l4[(e >> 1) & 3] += p0 + p1;
+    pk[e / 2] = pack_bf16x2(p0, p1);
+  }
+  mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+  return (l4[0] + l4[1]) + (l4[2] + l4[3]);
+}
+
 __global__ void __launch_bounds__(kThreads, 1) masked_tc_kernel(const __grid_constant__ TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -569,23 +598,50 @@ __global__ void __launch_bounds__(kThreads, 1) masked_tc_kernel(const __grid_con
       tmem_ld32(lane_base + colS + 64, s + 64);
       tmem_ld32(lane_base + colS + 96, s + 96);
       tmem_wait_ld();
-      const float mh = full ? fmaxf(half_max<true>(s, 0, ra, wb, we), half_max<true>(s + kHalf, kHalf, ra, wb, we))
-                            : fmaxf(half_max<false>(s, 0, ra, wb, we), half_max<false>(s + kHalf, kHalf, ra, wb, we));
+      // Speculative pass (every row of the warp has a maximum in use): the
+      // exponentials against it, this tile's maximum alongside, P kept in
+      // registers; S is read again from TMEM and the pass redone with the new
+      // maximum only when some row's grew by more than 8 (log2).
+      float lt = 0.f, mh = -INFINITY;
+      bool redo = true;
+      if (__all_sync(0xffffffffu, m_ref != -INFINITY)) {
+        uint32_t pk0[kHalf / 2], pk1[kHalf / 2];
+        float mx0, mx1;
+        lt = full ? half_exp_max<true>(s, 0, ra, wb, we, p.scale_log2, m_ref, pk0, mx0)
+                  : half_exp_max<false>(s, 0, ra, wb, we, p.scale_log2, m_ref, pk0, mx0);
+        lt += full ? half_exp_max<true>(s + kHalf, kHalf, ra, wb, we, p.scale_log2, m_ref, pk1, mx1)
+                   : half_exp_max<false>(s + kHalf, kHalf, ra, wb, we, p.scale_log2, m_ref, pk1, mx1);
+        mh = fmaxf(mx0, mx1);
+        redo = __any_sync(0xffffffffu, mh * p.scale_log2 > m_ref + 8.f);
+        if (!redo) {
+          tmem_st_pairs(lane_base + colS, pk0);
+          tmem_st_pairs(lane_base + colS + kHalf / 2, pk1);
+        }
+      } else {
+        mh = full ? fmaxf(half_max<true>(s, 0, ra, wb, we), half_max<true>(s + kHalf, kHalf, ra, wb, we))
+                  : fmaxf(half_max<false>(s, 0, ra, wb, we), half_max<false>(s + kHalf, kHalf, ra, wb, we));
+      }
       if (stamp) TC_CYC(j, 2);
       // lazy rescale: only when the max (log2 units) grew by more than 8
       const float mt_s = mh * p.scale_log2;
-      const bool grow = mt_s > m_ref + 8.f;
+      const bool grow = redo && mt_s > m_ref + 8.f;
       const float m_new = grow ? mt_s : m_ref;
       const float corr = grow ? ex2(m_ref - m_new) : 1.f;  // 0 when m_ref was -inf
       const float msub = (m_new == -INFINITY) ? 0.f : m_new;
-      // pass 2: exponentials; P (bf16 pairs) goes over S columns [0, 64)
-      float lt = 0.f;
-#pragma unroll
-      for (int c0 = 0; c0 < kTile; c0 += kHalf) {
-        uint32_t pk[kHalf / 2];
-        lt += full ? half_exp<true>(s + c0, c0, ra, wb, we, p.scale_log2, msub, pk)
-                   : half_exp<false>(s + c0, c0, ra, wb, we, p.scale_log2, msub, pk);
-        tmem_st_pairs(lane_base + colS + c0 / 2, pk);
+      if (redo) {
+        // pass 2: exponentials; P (bf16 pairs) goes over S columns [0, 64)
+        lt = 0.f;
+#pragma unroll 1
+        for (int c0 = 0; c0 < kTile; c0 += kHalf) {
+          float s2[kHalf];
+          tmem_ld32(lane_base + colS + c0, s2);
+          tmem_ld32(lane_base + colS + c0 + 32, s2 + 32);
+          tmem_wait_ld();
+          uint32_t pk[kHalf / 2];
+          lt += full ? half_exp<true>(s2, c0, ra, wb, we, p.scale_log2, msub, pk)
+                     : half_exp<false>(s2, c0, ra, wb, we, p.scale_log2, msub, pk);
+          tmem_st_pairs(lane_base + colS + c0 / 2, pk);
+        }
       }
       if (stamp) TC_CYC(j, 3);
       // O_g was last written by PV_g(j-1), complete before S_g(j) was signalled
