@@ -23,9 +23,10 @@
 //   into a 2-stage ring freed by the PV MMAs.  Warp 1 owns the tensor memory
 //   (512 columns: S_a, S_b, O_a, O_b) and one lane issues the MMAs.
 // * Warps 2-5 run the softmax of query tile a, warps 6-9 that of tile b, one
-//   thread per query row (TMEM lane): it reads its 128 scores with
-//   tcgen05.ld (two passes of 64 columns: maximum, then exponentials), forms
-//   p = 2^(s*scale*log2e - m), and writes P (bf16 pairs) over the first 64
+//   thread per query row (TMEM lane): it reads its 128 scores into registers
+//   with tcgen05.ld, forms p = 2^(s*scale*log2e - m) in one pass against the
+//   maximum in use (redone with the new maximum only when the row's maximum
+//   grew by more than 2^8), and writes P (bf16 pairs) over the first 64
 //   columns of its S with tcgen05.st.  The PV MMA reads P from TMEM.
 // * Issue order per key tile j: PV_a(j), S_a(j+1), PV_b(j), S_b(j+1).  While
 //   one group computes exponentials, the tensor core runs the other group's
