@@ -25,9 +25,10 @@
 // * Warps 2-5 run the softmax of query tile a, warps 6-9 that of tile b, one
 //   thread per query row (TMEM lane): it reads its 128 scores into registers
 //   with tcgen05.ld, forms p = 2^(s*scale*log2e - m) in one pass against the
-//   maximum in use (redone with the new maximum only when the row's maximum
-//   grew by more than 2^8), and writes P (bf16 pairs) over the first 64
-//   columns of its S with tcgen05.st.  The PV MMA reads P from TMEM.
+//   maximum in use, and writes P (bf16 pairs) over the first 64 columns of
+//   its S with tcgen05.st.  The PV MMA reads P from TMEM.  A row sum of at
+//   most 2^8 bounds every weight by 2^8, so the row maximum is only taken
+//   (and the pass redone) when some row's sum exceeds it.
 // * Issue order per key tile j: PV_a(j), S_a(j+1), PV_b(j), S_b(j+1).  While
 //   one group computes exponentials, the tensor core runs the other group's
 //   products, and vice versa.  S_g(j+1) overwrites P_g(j) only after PV_g(j)
@@ -332,35 +333,6 @@ __device__ __forceinline__ float half_exp(const float* s, int col0, int ra, int 
   return (l4[0] + l4[1]) + (l4[2] + l4[3]);
 }
 
-// half_exp that also returns the maximum of the visible raw scores (for the
-// speculative pass: the exponentials use the maximum in use, and this tile's
-// maximum only decides whether the pass must be redone).
-template <bool FULL>
-__device__ __forceinline__ float half_exp_max(const float* s, int col0, int ra, int wb, int we, float sl2, float msub,
-                                              uint32_t* pk, float& mx) {
-  float l4[4] = {0.f, 0.f, 0.f, 0.f};
-  float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-  for (int e = 0; e < kHalf; e += 2) {
-    const int c = col0 + e;
-    float x0 = fmaf(s[e], sl2, -msub), x1 = fmaf(s[e + 1], sl2, -msub);
-    float s0 = s[e], s1 = s[e + 1];
-    if (!FULL) {
-      const bool v0 = c < ra || (c >= wb && c <= we), v1 = c + 1 < ra || (c + 1 >= wb && c + 1 <= we);
-      x0 = v0 ? x0 : -INFINITY;
-      x1 = v1 ? x1 : -INFINITY;
-      s0 = v0 ? s0 : -INFINITY;
-      s1 = v1 ? s1 : -INFINITY;
-    }
-    m4[(e >> 1) & 3] = max3(m4[(e >> 1) & 3], s0, s1);
-    const float p0 = ex2(x0), p1 = ex2(x1);
-    l4[(e >> 1) & 3] += p0 + p1;
-    pk[e / 2] = pack_bf16x2(p0, p1);
-  }
-  mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-  return (l4[0] + l4[1]) + (l4[2] + l4[3]);
-}
-
 __global__ void __launch_bounds__(kThreads, 1) masked_tc_kernel(const __grid_constant__ TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -591,8 +563,7 @@ __global__ void __launch_bounds__(kThreads, 1) masked_tc_kernel(const __grid_con
           we = i - k0;
         }
       }
-      // the 128 scores into registers once: pass 1 (maximum) and pass 2
-      // (exponentials) read them there
+      // the 128 scores into registers once
       float s[kTile];
       tmem_ld32(lane_base + colS, s);
       tmem_ld32(lane_base + colS + 32, s + 32);
@@ -600,23 +571,32 @@ __global__ void __launch_bounds__(kThreads, 1) masked_tc_kernel(const __grid_con
       tmem_ld32(lane_base + colS + 96, s + 96);
       tmem_wait_ld();
       // Speculative pass (every row of the warp has a maximum in use): the
-      // exponentials against it, this tile's maximum alongside, P kept in
-      // registers; S is read again from TMEM and the pass redone with the new
-      // maximum only when some row's grew by more than 8 (log2).
+      // exponentials against it, P kept in registers.  A row sum of at most
+      // 2^8 bounds every weight by 2^8, so the maximum in use stands and no
+      // row maximum is needed; otherwise S is read again from TMEM, its
+      // maximum taken and the pass redone (with the new maximum when it grew
+      // by more than 8, log2).
       float lt = 0.f, mh = -INFINITY;
       bool redo = true;
       if (__all_sync(0xffffffffu, m_ref != -INFINITY)) {
         uint32_t pk0[kHalf / 2], pk1[kHalf / 2];
-        float mx0, mx1;
-        lt = full ? half_exp_max<true>(s, 0, ra, wb, we, p.scale_log2, m_ref, pk0, mx0)
-                  : half_exp_max<false>(s, 0, ra, wb, we, p.scale_log2, m_ref, pk0, mx0);
-        lt += full ? half_exp_max<true>(s + kHalf, kHalf, ra, wb, we, p.scale_log2, m_ref, pk1, mx1)
-                   : half_exp_max<false>(s + kHalf, kHalf, ra, wb, we, p.scale_log2, m_ref, pk1, mx1);
-        mh = fmaxf(mx0, mx1);
-        redo = __any_sync(0xffffffffu, mh * p.scale_log2 > m_ref + 8.f);
+        lt = full ? half_exp<true>(s, 0, ra, wb, we, p.scale_log2, m_ref, pk0)
+                  : half_exp<false>(s, 0, ra, wb, we, p.scale_log2, m_ref, pk0);
+        lt += full ? half_exp<true>(s + kHalf, kHalf, ra, wb, we, p.scale_log2, m_ref, pk1)
+                   : half_exp<false>(s + kHalf, kHalf, ra, wb, we, p.scale_log2, m_ref, pk1);
+        redo = __any_sync(0xffffffffu, !(lt <= 256.f));
         if (!redo) {
           tmem_st_pairs(lane_base + colS, pk0);
           tmem_st_pairs(lane_base + colS + kHalf / 2, pk1);
+        } else {
+#pragma unroll 1
+          for (int c0 = 0; c0 < kTile; c0 += kHalf) {
+            float s2[kHalf];
+            tmem_ld32(lane_base + colS + c0, s2);
+            tmem_ld32(lane_base + colS + c0 + 32, s2 + 32);
+            tmem_wait_ld();
+            mh = fmaxf(mh, full ? half_max<true>(s2, c0, ra, wb, we) : half_max<false>(s2, c0, ra, wb, we));
+          }
         }
       } else {
         mh = full ? fmaxf(half_max<true>(s, 0, ra, wb, we), half_max<true>(s + kHalf, kHalf, ra, wb, we))
