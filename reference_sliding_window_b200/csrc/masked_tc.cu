@@ -314,23 +314,46 @@ __device__ __forceinline__ float half_max(const float* s, int col0, int ra, int 
 // Exponentials p = 2^(s*sl2 - msub) of those 64 columns, one XU
 // instruction each, packed to bf16 pairs (the PV product's operand); returns
 // their float32 sum.  Masked columns get an argument of -inf, so exactly 0.
+// Fully visible tiles form two arguments with one fma.rn.f32x2 and add two
+// weights to the sums with one add.rn.f32x2 (the same roundings per element).
 template <bool FULL>
 __device__ __forceinline__ float half_exp(const float* s, int col0, int ra, int wb, int we, float sl2, float msub,
                                           uint32_t* pk) {
-  float l4[4] = {0.f, 0.f, 0.f, 0.f};  // independent sums
+  if constexpr (FULL) {
+    unsigned long long acc[2] = {0ull, 0ull};  // two pairs of independent sums
+    unsigned long long sl2x2, nmx2;
+    asm("mov.b64 %0, {%1, %1};" : "=l"(sl2x2) : "f"(sl2));
+    asm("mov.b64 %0, {%1, %1};" : "=l"(nmx2) : "f"(-msub));
 #pragma unroll
-  for (int e = 0; e < kHalf; e += 2) {
-    const int c = col0 + e;
-    float x0 = fmaf(s[e], sl2, -msub), x1 = fmaf(s[e + 1], sl2, -msub);
-    if (!FULL) {
+    for (int e = 0; e < kHalf; e += 2) {
+      unsigned long long sx, xx, pp;
+      asm("mov.b64 %0, {%1, %2};" : "=l"(sx) : "f"(s[e]), "f"(s[e + 1]));
+      asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(xx) : "l"(sx), "l"(sl2x2), "l"(nmx2));
+      float x0, x1;
+      asm("mov.b64 {%0, %1}, %2;" : "=f"(x0), "=f"(x1) : "l"(xx));
+      const float p0 = ex2(x0), p1 = ex2(x1);
+      asm("mov.b64 %0, {%1, %2};" : "=l"(pp) : "f"(p0), "f"(p1));
+      asm("add.rn.f32x2 %0, %0, %1;" : "+l"(acc[(e >> 1) & 1]) : "l"(pp));
+      pk[e / 2] = pack_bf16x2(p0, p1);
+    }
+    float a0, a1, b0, b1;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(acc[0]));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(b0), "=f"(b1) : "l"(acc[1]));
+    return (a0 + a1) + (b0 + b1);
+  } else {
+    float l4[4] = {0.f, 0.f, 0.f, 0.f};  // independent sums
+#pragma unroll
+    for (int e = 0; e < kHalf; e += 2) {
+      const int c = col0 + e;
+      float x0 = fmaf(s[e], sl2, -msub), x1 = fmaf(s[e + 1], sl2, -msub);
       x0 = (c < ra || (c >= wb && c <= we)) ? x0 : -INFINITY;
       x1 = (c + 1 < ra || (c + 1 >= wb && c + 1 <= we)) ? x1 : -INFINITY;
+      const float p0 = ex2(x0), p1 = ex2(x1);
+      l4[(e >> 1) & 3] += p0 + p1;
+      pk[e / 2] = pack_bf16x2(p0, p1);
     }
-    const float p0 = ex2(x0), p1 = ex2(x1);
-    l4[(e >> 1) & 3] += p0 + p1;
-    pk[e / 2] = pack_bf16x2(p0, p1);
+    return (l4[0] + l4[1]) + (l4[2] + l4[3]);
   }
-  return (l4[0] + l4[1]) + (l4[2] + l4[3]);
 }
 
 __global__ void __launch_bounds__(kThreads, 1) masked_tc_kernel(const __grid_constant__ TcParams p) {
