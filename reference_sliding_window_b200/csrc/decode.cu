@@ -126,6 +126,14 @@ struct DecTraits {
 
 __device__ __forceinline__ int ld_cg(const int32_t* p) { return __ldcg(p); }
 
+// 2^x by the XU instruction (arguments here are at most 8; results below
+// 2^-126 flush to zero, negligible beside the weight of the running maximum).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // RSWA_TIMING builds record %globaltimer stamps per CTA (profiling aid).
 #ifdef RSWA_TIMING
 #define RSWA_STAMP(k) \
@@ -731,19 +739,21 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
         const float sc = valid ? (kMixed ? part[0] * p.scale_log2 : part[0]) : -INFINITY;
         // Lazy running maximum: exponents stay <= 2^8 over the maximum in use,
         // so the maximum is reduced (and o, l rescaled) only when a score
-        // exceeds it by more than 8 (always on a warp's first part).
+        // exceeds it by more than 8.  A warp's first maximum in use is the
+        // score of the part's row 0 (valid here), not a reduction.
+        if (m == -INFINITY) m = __shfl_sync(0xffffffffu, sc, 0);
         if (__any_sync(0xffffffffu, sc > m + 8.f)) {
           float mx = sc;
 #pragma unroll
           for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
           const float m_new = fmaxf(m, mx);  // finite: the stage has a valid row
-          const float corr = exp2f(m - m_new);
+          const float corr = ex2_approx(m - m_new);
           l *= corr;
 #pragma unroll
           for (int e = 0; e < EPV; ++e) of[e] *= corr;
           m = m_new;
         }
-        const float pr = valid ? exp2f(sc - m) : 0.f;
+        const float pr = valid ? ex2_approx(sc - m) : 0.f;
         l += owner ? pr : 0.f;
         if (gs == 0 && lane == 0) RSWA_CYC(5);
         uint4 vu[NV];
