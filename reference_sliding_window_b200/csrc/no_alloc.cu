@@ -37,7 +37,7 @@ constexpr int kNoAllocMaxD = 128;
 
 // Scratch layout (bytes), every region 256-byte aligned.
 constexpr size_t kNaErr = 0;                                       // int32 error word
-constexpr size_t kNaDone = 4;                                      // unused (zeroed with the counter)
+constexpr size_t kNaZeroed = 4;                                    // [4, kNaLm) is zeroed before each launch
 constexpr size_t kNaT = 256;                                       // int32 step counter (always 0)
 constexpr size_t kNaLm = 512;                                      // int32[max slabs]
 constexpr size_t kNaTickets = kNaLm + 4 * kNoAllocMaxSlabs;        // int32[max slabs]
@@ -160,9 +160,9 @@ extern "C" rswa_status rswa_decode_noalloc(const void* k_cache, const void* v_ca
   g_na_begin[G] = n_items;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // Counters and tickets must start at zero (the error word is kept for
-  // rswa_decode_noalloc_check); plan and lengths are uploaded.
-  if (cudaMemsetAsync(scratch + kNaDone, 0, kNaLm - kNaDone, s) != cudaSuccess ||
+  // The step counter and the tickets must start at zero (the error word is
+  // kept for rswa_decode_noalloc_check); plan and lengths are uploaded.
+  if (cudaMemsetAsync(scratch + kNaZeroed, 0, kNaLm - kNaZeroed, s) != cudaSuccess ||
       cudaMemsetAsync(scratch + kNaTickets, 0, 4 * (size_t)nbh, s) != cudaSuccess ||
       cudaMemcpyAsync(scratch + kNaLm, g_na_lens, 4 * (size_t)batch, cudaMemcpyHostToDevice, s) != cudaSuccess ||
       cudaMemcpyAsync(scratch + kNaItems, g_na_items, sizeof(DecodeItem) * n_items, cudaMemcpyHostToDevice, s) !=
